@@ -1,0 +1,247 @@
+"""Thin ctypes binding of libsmc (C ABI in include/smc.h).
+
+Every function here only marshals arguments: it checks tensor properties,
+takes raw device pointers and the current CUDA stream from PyTorch, and calls
+the C entry point of the same name.  All computation runs in libsmc's CUDA
+kernels; there is no CPU path.  Importing works without a GPU (so the symbol
+table can be checked anywhere); calls need the CUDA device the tensors live on.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsmc.so")
+
+SMC_OK = 0
+STATUS = {
+    0: "SMC_OK", -1: "SMC_ERR_INVALID", -2: "SMC_ERR_DUPLICATE", -3: "SMC_ERR_RANGE",
+    -4: "SMC_ERR_OOM", -5: "SMC_ERR_CUDA", -6: "SMC_ERR_UNSUPPORTED", -7: "SMC_ERR_TABLE_FULL",
+    -8: "SMC_ERR_TIMEOUT",
+}
+DTYPE_CODE = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
+ORDER_CODE = {"mask": 0, "input": 1}
+
+# every symbol include/smc.h declares
+EXPORTS = (
+    "smc_build_index", "smc_build_index_ex", "smc_forward", "smc_get_neighbor_map",
+    "smc_get_plan_stats", "smc_get_sizes", "smc_get_tile_plan", "smc_device_status",
+    "smc_destroy", "smc_status_string", "smc_version",
+)
+
+
+class SmcError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({status_string(status)})")
+
+
+class _Options(ctypes.Structure):
+    _fields_ = [("table_capacity", ctypes.c_int64), ("order", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libsmc.so; raises if the library has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"libsmc.so not found at {LIB_PATH}; build it with "
+            "`python -m submanifold_sparse_convolution_coord_b200.csrc.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    p, i64, i32, i = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int
+    L.smc_build_index.argtypes = [p, i64, i32, ctypes.POINTER(p)]
+    L.smc_build_index_ex.argtypes = [p, i64, i32, ctypes.POINTER(_Options), p, ctypes.POINTER(p)]
+    L.smc_forward.argtypes = [p, p, p, p, i, i, i, i, p]
+    L.smc_get_neighbor_map.argtypes = [p, p, p]
+    L.smc_get_plan_stats.argtypes = [p, ctypes.POINTER(i64), ctypes.POINTER(i64)]
+    L.smc_get_sizes.argtypes = [p, ctypes.POINTER(i64), ctypes.POINTER(i64)]
+    L.smc_get_tile_plan.argtypes = [p, p, p, p]
+    L.smc_device_status.argtypes = [p, p]
+    L.smc_destroy.argtypes = [p]
+    L.smc_destroy.restype = None
+    L.smc_status_string.argtypes = [i]
+    L.smc_status_string.restype = ctypes.c_char_p
+    L.smc_version.argtypes = []
+    for name in EXPORTS:
+        fn = getattr(L, name)
+        if name not in ("smc_destroy", "smc_status_string"):
+            fn.restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def status_string(status: int) -> str:
+    return lib().smc_status_string(int(status)).decode()
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != SMC_OK:
+        raise SmcError(rc, where)
+
+
+def _stream(stream: Optional[torch.cuda.Stream], device: torch.device) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dev_ptr(t: torch.Tensor, name: str, dtype=None) -> int:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+# ----------------------------------------------------------------------------
+# same-name wrappers
+# ----------------------------------------------------------------------------
+def smc_build_index(coords: torch.Tensor, stride: int = 1, table_capacity: int = 0,
+                    order: str = "mask", stream: Optional[torch.cuda.Stream] = None) -> int:
+    """coords: CUDA int32 [N, 4] (b, x, y, z).  Returns the raw handle (int)."""
+    if coords.dim() != 2 or coords.shape[1] != 4:
+        raise ValueError("coords must be [N, 4]")
+    ptr = _dev_ptr(coords, "coords", torch.int32)
+    opts = _Options(int(table_capacity), ORDER_CODE[order], 0)
+    h = ctypes.c_void_p()
+    rc = lib().smc_build_index_ex(ctypes.c_void_p(ptr), coords.shape[0], int(stride),
+                                  ctypes.byref(opts), _stream(stream, coords.device),
+                                  ctypes.byref(h))
+    _check(rc, "smc_build_index")
+    return h.value
+
+
+def smc_forward(handle: int, feats: torch.Tensor, W: torch.Tensor, out: torch.Tensor, K: int,
+                cin: int, cout: int, stream: Optional[torch.cuda.Stream] = None) -> None:
+    dtype = feats.dtype
+    if dtype not in DTYPE_CODE:
+        raise ValueError(f"unsupported dtype {dtype}")
+    fp = _dev_ptr(feats, "feats", dtype)
+    wp = _dev_ptr(W, "W", dtype)
+    op = _dev_ptr(out, "out", dtype)
+    rc = lib().smc_forward(ctypes.c_void_p(handle), ctypes.c_void_p(fp), ctypes.c_void_p(wp),
+                           ctypes.c_void_p(op), int(K), int(cin), int(cout), DTYPE_CODE[dtype],
+                           _stream(stream, feats.device))
+    _check(rc, "smc_forward")
+
+
+def smc_get_neighbor_map(handle: int, map_out: torch.Tensor,
+                         stream: Optional[torch.cuda.Stream] = None) -> None:
+    rc = lib().smc_get_neighbor_map(ctypes.c_void_p(handle),
+                                    ctypes.c_void_p(_dev_ptr(map_out, "map", torch.int32)),
+                                    _stream(stream, map_out.device))
+    _check(rc, "smc_get_neighbor_map")
+
+
+def smc_get_plan_stats(handle: int) -> tuple:
+    u, s = ctypes.c_int64(), ctypes.c_int64()
+    _check(lib().smc_get_plan_stats(ctypes.c_void_p(handle), ctypes.byref(u), ctypes.byref(s)),
+           "smc_get_plan_stats")
+    return u.value, s.value
+
+
+def smc_get_sizes(handle: int) -> tuple:
+    n, t = ctypes.c_int64(), ctypes.c_int64()
+    _check(lib().smc_get_sizes(ctypes.c_void_p(handle), ctypes.byref(n), ctypes.byref(t)),
+           "smc_get_sizes")
+    return n.value, t.value
+
+
+def smc_get_tile_plan(handle: int, perm: Optional[torch.Tensor], tile_mask: Optional[torch.Tensor],
+                      stream: Optional[torch.cuda.Stream] = None) -> None:
+    dev = (perm if perm is not None else tile_mask).device
+    pp = _dev_ptr(perm, "perm", torch.int32) if perm is not None else None
+    mp = _dev_ptr(tile_mask, "tile_mask", torch.int32) if tile_mask is not None else None
+    rc = lib().smc_get_tile_plan(ctypes.c_void_p(handle), ctypes.c_void_p(pp),
+                                 ctypes.c_void_p(mp), _stream(stream, dev))
+    _check(rc, "smc_get_tile_plan")
+
+
+def smc_device_status(handle: int, device=None, stream: Optional[torch.cuda.Stream] = None) -> int:
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    return lib().smc_device_status(ctypes.c_void_p(handle), _stream(stream, dev))
+
+
+def smc_destroy(handle: int) -> None:
+    if handle:
+        lib().smc_destroy(ctypes.c_void_p(handle))
+
+
+def smc_version() -> int:
+    return lib().smc_version()
+
+
+# ----------------------------------------------------------------------------
+# convenience object
+# ----------------------------------------------------------------------------
+class SubMIndex:
+    """Owns one handle: the neighbour map and tile plan of a coordinate set
+    (the cached indice map of the README's SparseTensor)."""
+
+    def __init__(self, coords: torch.Tensor, stride: int = 1, table_capacity: int = 0,
+                 order: str = "mask"):
+        self.device = coords.device
+        self.handle = smc_build_index(coords, stride, table_capacity, order)
+        self.n, self.n_tiles = smc_get_sizes(self.handle)
+
+    def close(self) -> None:
+        if getattr(self, "handle", None):
+            smc_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    def neighbor_map(self) -> torch.Tensor:
+        out = torch.empty((self.n, 27), dtype=torch.int32, device=self.device)
+        smc_get_neighbor_map(self.handle, out)
+        return out
+
+    def plan_stats(self) -> tuple:
+        return smc_get_plan_stats(self.handle)
+
+    def tile_plan(self) -> tuple:
+        perm = torch.empty(self.n, dtype=torch.int32, device=self.device)
+        tmask = torch.empty(self.n_tiles, dtype=torch.int32, device=self.device)
+        smc_get_tile_plan(self.handle, perm, tmask)
+        return perm, tmask
+
+    def status(self) -> int:
+        return smc_device_status(self.handle, self.device)
+
+    def forward(self, feats: torch.Tensor, W: torch.Tensor, K: int = 3,
+                out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        if feats.dim() != 2 or feats.shape[0] != self.n:
+            raise ValueError("feats must be [N, Cin] for this index")
+        taps, cin, cout = W.shape
+        if taps != K ** 3 or cin != feats.shape[1]:
+            raise ValueError("W must be [K^3, Cin, Cout]")
+        if out is None:
+            out = torch.empty((self.n, cout), dtype=feats.dtype, device=feats.device)
+        smc_forward(self.handle, feats, W, out, K, cin, cout)
+        return out
+
+
+def submconv3d(index: SubMIndex, feats: torch.Tensor, W: torch.Tensor, K: int = 3,
+               out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    return index.forward(feats, W, K, out)

@@ -1,0 +1,180 @@
+// C ABI of libsmc (declared in include/smc.h): argument checks, the index
+// handle and dispatch to the kernels.  No call here touches the CPU copy of
+// any tensor, and no compute path exists outside the CUDA kernels.
+#include <cstdint>
+#include <new>
+
+#include "smc_internal.h"
+
+struct smc_index {
+  int device = 0;
+  int32_t stride = 1;
+  smc::Plan plan;
+};
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int elem_bytes(int dtype) {
+  switch (dtype) {
+    case SMC_F32:
+      return 4;
+    case SMC_F16:
+    case SMC_BF16:
+      return 2;
+    default:
+      return 0;
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+int smc_version(void) { return 100; }
+
+const char* smc_status_string(int status) {
+  switch (status) {
+    case SMC_OK:
+      return "ok";
+    case SMC_ERR_INVALID:
+      return "invalid argument";
+    case SMC_ERR_DUPLICATE:
+      return "duplicate coordinate";
+    case SMC_ERR_RANGE:
+      return "coordinate out of range (b in [0,32768), x,y,z in [0,65536))";
+    case SMC_ERR_OOM:
+      return "device allocation failed";
+    case SMC_ERR_CUDA:
+      return "CUDA error";
+    case SMC_ERR_UNSUPPORTED:
+      return "unsupported shape or dtype";
+    case SMC_ERR_TABLE_FULL:
+      return "coordinate hash table full";
+    case SMC_ERR_TIMEOUT:
+      return "a device-side wait timed out";
+    default:
+      return "unknown status";
+  }
+}
+
+int smc_build_index_ex(const int32_t* coords_dev, int64_t n, int32_t stride,
+                       const smc_index_options* opts, smc_stream_t stream,
+                       smc_handle_t* out_handle) {
+  if (!out_handle) return SMC_ERR_INVALID;
+  *out_handle = nullptr;
+  if (n < 0 || stride < 1 || (n > 0 && !coords_dev)) return SMC_ERR_INVALID;
+  if (n > 0 && !aligned16(coords_dev)) return SMC_ERR_INVALID;
+  if (n >= (int64_t(1) << 31) / smc::kTaps) return SMC_ERR_UNSUPPORTED;
+  int64_t cap = 0;
+  int32_t order = SMC_ORDER_MASK;
+  if (opts) {
+    if (opts->reserved != 0 || opts->table_capacity < 0 ||
+        (opts->order != SMC_ORDER_MASK && opts->order != SMC_ORDER_INPUT))
+      return SMC_ERR_INVALID;
+    cap = opts->table_capacity;
+    order = opts->order;
+  }
+  smc_index* h = new (std::nothrow) smc_index();
+  if (!h) return SMC_ERR_OOM;
+  if (cudaGetDevice(&h->device) != cudaSuccess) {
+    delete h;
+    return SMC_ERR_CUDA;
+  }
+  h->stride = stride;
+  const int rc = smc::build_plan(coords_dev, n, stride, cap, order,
+                                 reinterpret_cast<cudaStream_t>(stream), &h->plan);
+  if (rc != SMC_OK) {
+    delete h;
+    return rc;
+  }
+  *out_handle = h;
+  return SMC_OK;
+}
+
+int smc_build_index(const int32_t* coords_dev, int64_t n, int32_t stride,
+                    smc_handle_t* out_handle) {
+  return smc_build_index_ex(coords_dev, n, stride, nullptr, nullptr, out_handle);
+}
+
+int smc_forward(smc_handle_t h, const void* feats, const void* W, void* out, int K, int cin,
+                int cout, int dtype, smc_stream_t stream) {
+  if (!h) return SMC_ERR_INVALID;
+  if (K != 1 && K != 3) return SMC_ERR_INVALID;
+  if (elem_bytes(dtype) == 0 || cin < 1 || cout < 1) return SMC_ERR_INVALID;
+  const smc::Plan& plan = h->plan;
+  if (plan.n == 0) return SMC_OK;
+  if (!feats || !W || !out) return SMC_ERR_INVALID;
+  if (!aligned16(feats) || !aligned16(W) || !aligned16(out)) return SMC_ERR_INVALID;
+  const bool dense = (K == 1);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (smc::conv_tc_supported(cin, cout, dtype))
+    return smc::launch_conv_tc(plan, dense, feats, W, out, cin, cout, dtype, s);
+  return smc::launch_conv_simt(plan, dense, feats, W, out, cin, cout, dtype, s);
+}
+
+int smc_get_neighbor_map(smc_handle_t h, int32_t* map_dev, smc_stream_t stream) {
+  if (!h) return SMC_ERR_INVALID;
+  if (h->plan.n == 0) return SMC_OK;
+  if (!map_dev) return SMC_ERR_INVALID;
+  return cudaMemcpyAsync(map_dev, h->plan.nbr, size_t(h->plan.n) * smc::kTaps * sizeof(int32_t),
+                         cudaMemcpyDeviceToDevice,
+                         reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? SMC_OK
+             : SMC_ERR_CUDA;
+}
+
+int smc_get_plan_stats(smc_handle_t h, int64_t* useful_pairs, int64_t* issued_rows_taps) {
+  if (!h) return SMC_ERR_INVALID;
+  if (useful_pairs) *useful_pairs = h->plan.useful_pairs;
+  if (issued_rows_taps) *issued_rows_taps = h->plan.issued_rows_taps;
+  return SMC_OK;
+}
+
+int smc_get_sizes(smc_handle_t h, int64_t* n, int64_t* n_tiles) {
+  if (!h) return SMC_ERR_INVALID;
+  if (n) *n = h->plan.n;
+  if (n_tiles) *n_tiles = h->plan.n_tiles;
+  return SMC_OK;
+}
+
+int smc_get_tile_plan(smc_handle_t h, int32_t* perm_dev, uint32_t* tile_mask_dev,
+                      smc_stream_t stream) {
+  if (!h) return SMC_ERR_INVALID;
+  const smc::Plan& p = h->plan;
+  if (p.n == 0) return SMC_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (perm_dev && cudaMemcpyAsync(perm_dev, p.perm, size_t(p.n) * sizeof(int32_t),
+                                  cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return SMC_ERR_CUDA;
+  if (tile_mask_dev && cudaMemcpyAsync(tile_mask_dev, p.tile_mask, size_t(p.n_tiles) * sizeof(uint32_t),
+                                       cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return SMC_ERR_CUDA;
+  return SMC_OK;
+}
+
+int smc_device_status(smc_handle_t h, smc_stream_t stream) {
+  if (!h) return SMC_ERR_INVALID;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  if (cudaMemcpyAsync(&v, h->plan.status, sizeof(v), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return SMC_ERR_CUDA;
+  if (v != 0 && cudaMemsetAsync(h->plan.status, 0, sizeof(int32_t), s) != cudaSuccess)
+    return SMC_ERR_CUDA;
+  if (v & smc::kDevTimeout) return SMC_ERR_TIMEOUT;
+  return v == 0 ? SMC_OK : SMC_ERR_CUDA;
+}
+
+void smc_destroy(smc_handle_t h) {
+  if (!h) return;
+  int cur = 0;
+  cudaGetDevice(&cur);
+  if (cur != h->device) cudaSetDevice(h->device);
+  smc::free_plan(&h->plan);
+  if (cur != h->device) cudaSetDevice(cur);
+  delete h;
+}
+
+}  // extern "C"
