@@ -3,7 +3,11 @@
 Tolerances (the bar each parity test applies):
 
 * fp16 / bf16 features, fp32 accumulation, output in the feature dtype:
-  |out - ref| <= 2e-3 * S element-wise, S = sum_d |feats[c+d]| @ |W[d]|;
+  |out - ref| <= 2e-3 * S + u * |ref| element-wise, S = sum_d |feats[c+d]| @
+  |W[d]|.  2e-3 * S bounds the products and the fp32 accumulation; u * |ref|
+  is the one rounding of the stored result to the output dtype (unit
+  roundoff u = 2^-11 for fp16, 2^-8 for bf16), which 2e-3 * S alone does not
+  cover for bf16 when |ref| > 0.51 S (few-term sums, e.g. isolated voxels);
 * fp32 features: |out - ref| <= 1e-5 * |ref| + 1e-12 * S element-wise
   (the CUDA-core kernel accumulates in fp64 and rounds once to fp32).
 
@@ -16,6 +20,7 @@ import torch
 from oracle import native
 
 HALF_TOL = 2e-3
+UNIT_ROUNDOFF = {torch.float16: 2.0 ** -11, torch.bfloat16: 2.0 ** -8}
 F32_RTOL = 1e-5
 F32_FLOOR = 1e-12
 
@@ -32,7 +37,7 @@ def check_conv(out_gpu: torch.Tensor, ref: np.ndarray, scale: np.ndarray, what: 
     if out_gpu.dtype == torch.float32:
         bound = F32_RTOL * np.abs(ref) + F32_FLOOR * scale
     else:
-        bound = HALF_TOL * scale
+        bound = HALF_TOL * scale + UNIT_ROUNDOFF[out_gpu.dtype] * np.abs(ref)
     bad = err > bound
     if bad.any():
         idx = np.argwhere(bad)[:5]
