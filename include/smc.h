@@ -91,6 +91,39 @@ int smc_build_index_ex(const int32_t* coords_dev, int64_t n, int32_t stride,
                        const smc_index_options* opts, smc_stream_t stream,
                        smc_handle_t* out_handle);
 
+/* Largest n that smc_build_neighbor_map_static accepts. */
+#define SMC_STATIC_MAX_VOXELS 524288
+
+/*
+ * Neighbour map with no device allocation by the library.  The pages this
+ * library follows have no counterpart to this call; it exists for callers
+ * that may not allocate device memory themselves: code running inside a
+ * framework or server that reserves the GPU's memory up front and hands it out
+ * from its own pool (a cudaMalloc beside that pool fails under its cap or
+ * breaks its accounting), and latency-sensitive loops, where cudaMalloc and
+ * cudaFree may synchronise the device and stall other streams.
+ *
+ * coords_dev : device pointer, int32 [n][4] = (b, x, y, z), 16-byte aligned.
+ * n          : 0 <= n <= SMC_STATIC_MAX_VOXELS; a larger n returns
+ *              SMC_ERR_UNSUPPORTED and launches nothing.
+ * stride     : neighbour spacing, >= 1.
+ * map_dev    : device pointer, int32 [n][27], written like
+ *              smc_get_neighbor_map's output (-1 = no active neighbour).
+ * stream     : the work is queued on this stream, which the call then
+ *              synchronises to read the status word.
+ *
+ * Scratch: the coordinate hash table lives in one fixed array of static
+ * device memory (about 14 MiB), reserved on every GPU that loads libsmc and
+ * held until the process exits.  The first call on a device looks up that
+ * array's device address; make that first call before any stream capture.
+ * Every call, from any stream or host thread, uses the same array and clears
+ * the part it needs first, so calls that overlap on the GPU race with each
+ * other and must be serialised by the caller.
+ * Errors: SMC_ERR_INVALID, _UNSUPPORTED, _DUPLICATE, _RANGE, _CUDA.
+ */
+int smc_build_neighbor_map_static(const int32_t* coords_dev, int64_t n, int32_t stride,
+                                  int32_t* map_dev, smc_stream_t stream);
+
 /*
  * SubMConv3d forward over the handle's voxels.
  *

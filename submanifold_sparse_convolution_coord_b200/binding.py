@@ -30,7 +30,7 @@ ORDER_CODE = {"mask": 0, "input": 1}
 EXPORTS = (
     "smc_build_index", "smc_build_index_ex", "smc_forward", "smc_get_neighbor_map",
     "smc_get_plan_stats", "smc_get_sizes", "smc_get_tile_plan", "smc_device_status",
-    "smc_destroy", "smc_status_string", "smc_version",
+    "smc_destroy", "smc_status_string", "smc_version", "smc_build_neighbor_map_static",
 )
 
 
@@ -72,6 +72,7 @@ def lib() -> ctypes.CDLL:
     L.smc_status_string.argtypes = [i]
     L.smc_status_string.restype = ctypes.c_char_p
     L.smc_version.argtypes = []
+    L.smc_build_neighbor_map_static.argtypes = [p, i64, i32, p, p]
     for name in EXPORTS:
         fn = getattr(L, name)
         if name not in ("smc_destroy", "smc_status_string"):

@@ -463,3 +463,89 @@ int build_plan(const int32_t* coords, int64_t n, int32_t stride, int64_t table_c
 }
 
 }  // namespace smc
+
+// ---------------------------------------------------------------------------
+// Allocation-free neighbour map: smc_build_neighbor_map_static.
+//
+// For callers that may not allocate device memory themselves (see the header):
+// the same insert and query kernels as the index build above, with the hash
+// table in a fixed-size array of static device memory that every device
+// loading this library reserves once, for the life of the process.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+namespace smc {
+namespace {
+
+constexpr int64_t kStaticMaxVoxels = SMC_STATIC_MAX_VOXELS;
+constexpr int64_t kStaticSlots = 2 * kStaticMaxVoxels;  // load factor <= 1/2
+
+struct StaticScratch {
+  uint64_t keys[kStaticSlots];
+  int32_t vals[kStaticSlots];
+  uint32_t mask[kStaticMaxVoxels];
+  int32_t status;
+};
+
+// Host code may not use this name as a device address: the pointer passed to
+// the kernels comes from cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) StaticScratch g_static_scratch;
+
+constexpr int kMaxDevices = 128;
+std::mutex g_static_mutex;
+StaticScratch* g_static_ptr[kMaxDevices] = {};
+
+int static_scratch(StaticScratch** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return SMC_ERR_CUDA;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return SMC_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_static_mutex);
+  if (!g_static_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return SMC_ERR_CUDA;
+    }
+    g_static_ptr[dev] = static_cast<StaticScratch*>(p);
+  }
+  *out = g_static_ptr[dev];
+  return SMC_OK;
+}
+
+}  // namespace
+}  // namespace smc
+
+extern "C" int smc_build_neighbor_map_static(const int32_t* coords_dev, int64_t n, int32_t stride,
+                                             int32_t* map_dev, smc_stream_t stream) {
+  using namespace smc;
+  if (n < 0 || stride < 1) return SMC_ERR_INVALID;
+  if (n > kStaticMaxVoxels) return SMC_ERR_UNSUPPORTED;
+  if (n == 0) return SMC_OK;
+  if (!coords_dev || !map_dev) return SMC_ERR_INVALID;
+  if ((reinterpret_cast<uintptr_t>(coords_dev) & 15u) != 0) return SMC_ERR_INVALID;
+  StaticScratch* sc = nullptr;
+  int rc = static_scratch(&sc);
+  if (rc != SMC_OK) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint64_t cap = 64;
+  while (cap < uint64_t(2 * n)) cap <<= 1;
+  // The array keeps the previous call's contents: reset the slots this call
+  // probes and the status word before use.
+  if (cudaMemsetAsync(sc->keys, 0xFF, cap * sizeof(uint64_t), s) != cudaSuccess ||
+      cudaMemsetAsync(&sc->status, 0, sizeof(int32_t), s) != cudaSuccess)
+    return SMC_ERR_CUDA;
+  const int4* c4 = reinterpret_cast<const int4*>(coords_dev);
+  k_insert<<<grid_for(n, 256), 256, 0, s>>>(c4, n, sc->keys, sc->vals, cap - 1, &sc->status);
+  k_neighbors<<<grid_for(n, kNbrVoxels), kNbrThreads, 0, s>>>(c4, n, stride, sc->keys, sc->vals,
+                                                               cap - 1, map_dev, sc->mask);
+  if (cudaGetLastError() != cudaSuccess) return SMC_ERR_CUDA;
+  int32_t dev_status = 0;
+  if (cudaMemcpyAsync(&dev_status, &sc->status, sizeof(int32_t), cudaMemcpyDeviceToHost, s) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return SMC_ERR_CUDA;
+  return status_from_device(dev_status);
+}
