@@ -1,28 +1,44 @@
 // Output-stationary implicit-GEMM SubMConv3d on the sm_100a tensor cores.
 //
-// One CTA computes a 128-row x BN-column output tile.  For every tap the
-// tile's plan marks active (the others are skipped), the CTA gathers the 128
-// neighbour feature rows of that tap (zero rows for absent neighbours) and
-// multiplies them by W[tap] with tcgen05.mma, accumulating in fp32 in tensor
-// memory; each output row is then written exactly once, without atomics.
-// This is the sum over offsets of the trellis_sparse_mlx README ("What's in
-// it": out[c] = sum_d feats[c+d] @ W[d] over active neighbours) reorganised
-// so that the dense work the README's fused [N, 27 Cin] x [27 Cin, Cout]
-// matmul spends on absent neighbours is skipped a tile-tap at a time.
+// A work item is a 128-row x BN-column output tile.  For every tap the tile's
+// plan marks active (the others are skipped), the tile's 128 neighbour feature
+// rows of that tap are gathered into shared memory (zero rows for absent
+// neighbours) and multiplied by W[tap] with tcgen05.mma, accumulating in fp32
+// in tensor memory; each output row is then written exactly once, without
+// atomics.  This is the sum over offsets of the trellis_sparse_mlx README
+// ("What's in it": out[c] = sum_d feats[c+d] @ W[d] over active neighbours)
+// organised so that the dense work of the README's fused
+// [N, 27 Cin] x [27 Cin, Cout] matmul is skipped one tile-tap at a time.
 //
-// Warp roles (192 threads):
-//   warps 0-3  gather A: 16-byte cp.async copies of the neighbour rows into a
-//              128-byte-swizzled K-major tile (zero-filled for -1), then the
-//              epilogue (TMEM -> registers -> fp16/bf16 -> global);
-//   warp 4     lane 0 loads the W[tap] slice with TMA (MN-major, 128B swizzle);
-//   warp 5     allocates tensor memory; lane 0 issues the MMAs.
-// Stages are handed over with mbarriers; every wait is bounded in time and a
-// wait that runs out marks the CTA aborted and sets the status word.
+// Persistent kernel, one CTA per SM, 7 + 4 * STAGES warps:
+//   warp 0      lane 0 loads the W[tap] slice of each stage with TMA
+//               (MN-major, 128-byte swizzle);
+//   warp 1      allocates tensor memory; lane 0 issues the MMAs (M = 128,
+//               N = BN, K = 16) into one of two accumulators;
+//   warps 2-5   epilogue: tensor memory -> registers -> fp16/bf16 -> global,
+//               overlapping the MMAs of the next work item;
+//   warp 6      scheduler: takes work items (heaviest first) from a global
+//               counter and decodes each one's tile masks and slot offsets
+//               into a small shared-memory queue read by every other role;
+//   warps 7..   gather, four warps per pipeline stage slot: warp q of slot i
+//               copies rows 32 q .. 32 q + 31 of every tile the stage feeds
+//               (64 channels, 128 bytes per row) with 16-byte cp.async
+//               (zero-filled for absent neighbours) into a 128-byte-swizzled
+//               K-major tile; each lane's mbarrier arrival fires when its
+//               copies land, so no thread waits on its copies.  Many warps
+//               with few copies each keep enough copies in flight; fixed
+//               owners per slot keep every parity wait on a slot's barrier at
+//               most one phase ahead.
+// Stages and accumulators are handed over with mbarriers; every wait is
+// bounded in time and a wait that runs out marks the CTA aborted and sets the
+// status word, so a fault in the pipeline ends the kernel instead of hanging.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <algorithm>
+#include <cstdlib>
 #include <mutex>
 
 #include "smc_internal.h"
@@ -30,9 +46,14 @@
 namespace smc {
 namespace {
 
-constexpr int kThreads = 192;
-constexpr int kBK = 64;                        // input channels per stage (128 bytes)
-constexpr int kABytes = kTileRows * kBK * 2;   // 16 KB
+constexpr int kPrefetchWarp = 6;
+constexpr int kFirstGatherWarp = 7;
+constexpr int kWarpsPerSlot = 4;  // each copies 32 of a tile's 128 rows
+__host__ __device__ constexpr int threads_for(int stages) {
+  return 32 * (kFirstGatherWarp + kWarpsPerSlot * stages);
+}
+constexpr int kBK = 64;                          // input channels per stage (128 bytes)
+constexpr int kABytes = kTileRows * kBK * 2;     // 16 KB
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
 // ----------------------------------------------------------------------------
@@ -92,21 +113,6 @@ __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
   }
 }
 
-__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
-               "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-__device__ __forceinline__ void fence_async_proxy() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
                                             uint32_t bar) {
   asm volatile(
@@ -114,6 +120,17 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       "[%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
       : "memory");
+}
+// 16-byte copy global -> shared; src_bytes = 0 writes 16 zero bytes.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+// Arrive on `bar` once every cp.async this thread issued so far has landed
+// (the arrival is counted in the barrier's expected count).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -198,195 +215,385 @@ __device__ __forceinline__ uint32_t pack2(uint32_t a, uint32_t b) {
 struct ConvArgs {
   const uint16_t* feats;
   uint16_t* out;
-  const int32_t* gidx;
-  const int32_t* tile_off;
-  const uint8_t* tile_taps;
-  const int32_t* out_row;
+  const int32_t* gidx;        // [slots][128], -1 = absent
+  const int32_t* tile_off;    // [n_tiles + 1] first slot of each tile
+  const uint32_t* tile_mask;  // [n_tiles] active taps of each tile
+  const int32_t* out_row;     // [n_tiles * 128], -1 = padding row
+  uint32_t* work_counter;     // zeroed before the launch
   int32_t* status;
   int64_t n;
   int cin;
   int cout;
   int n_tiles;
-  int dense;
+  int n_groups;  // ceil(n_tiles / G)
+  int n_blocks;  // cout / BN
+  int dense;     // 1: K = 1, rows in order, one tap
 };
 
-template <int BN, int STAGES, int LAG, bool BF16>
-__global__ void __launch_bounds__(kThreads, 1)
+// A work item is a group of G consecutive tiles (in plan order) and one
+// BN-wide block of output channels.  The group's taps are the union of its
+// tiles' taps; a W chunk is loaded once per stage and multiplied into every
+// tile of the group that has that tap.  Items are numbered heaviest first and
+// handed out dynamically, so every SM stays busy until the end.
+template <int G>
+struct Group {
+  int w;         // item number, -1 = no more work
+  int tile0;
+  int n0;
+  uint32_t all;  // union of the masks
+  int rot;       // taps are visited starting at this tap (spreads W reads over L2)
+  uint32_t mask[G];
+  int slot0[G];  // first gather-index slot of each tile
+};
+
+template <int BN, int G>
+__device__ __forceinline__ Group<G> group_of(const ConvArgs& a, int w) {
+  Group<G> gr;
+  gr.w = w;
+  const int q = w / a.n_blocks;
+  gr.tile0 = (a.n_groups - 1 - q) * G;  // groups with the largest tap sets first
+  gr.n0 = (w - q * a.n_blocks) * BN;
+  gr.all = 0;
+#pragma unroll
+  for (int k = 0; k < G; ++k) {
+    const int t = gr.tile0 + k;
+    const bool live = t < a.n_tiles;
+    gr.mask[k] = live ? (a.dense ? 1u : a.tile_mask[t]) : 0u;
+    gr.slot0[k] = live && !a.dense ? a.tile_off[t] : 0;
+    gr.all |= gr.mask[k];
+  }
+  gr.rot = a.dense ? 0 : int((unsigned(w) * 7u) % unsigned(kTaps));
+  return gr;
+}
+
+// Taps of `all` in the order r, r+1, ..., 26, 0, ..., r-1 (set bits only).
+__device__ __forceinline__ uint32_t rotate_taps(uint32_t all, int r) {
+  constexpr uint32_t kAll = (1u << kTaps) - 1u;
+  return r == 0 ? all : (((all >> r) | (all << (kTaps - r))) & kAll);
+}
+__device__ __forceinline__ int next_tap(uint32_t& rotated, int r) {
+  const int b = __ffs(rotated) - 1;
+  rotated &= rotated - 1u;
+  const int t = b + r;
+  return t >= kTaps ? t - kTaps : t;
+}
+
+// One gather warp's share of a stage: which tiles it copies and from where.
+template <int G>
+struct GatherJob {
+  int stage;
+  uint32_t g;
+  int kb;
+  uint32_t tiles;  // bit k: tile k of the group has this tap
+  int vidx[G];     // lane l: source row of local row l of tile k (-1 = zero row)
+};
+
+constexpr int kQueue = 4;  // work items published ahead of the consumers
+
+template <int BN, int STAGES, int G, bool BF16>
+__global__ void __launch_bounds__(threads_for(STAGES), 1)
 k_conv_tc(const __grid_constant__ CUtensorMap wmap, const ConvArgs args) {
   static_assert(BN % 64 == 0 && BN <= 256, "BN");
-  static_assert(LAG >= 1 && LAG < STAGES, "LAG");
   constexpr int kBBytes = BN * kBK * 2;
-  constexpr int kStageBytes = kABytes + kBBytes;
-  constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
+  constexpr int kStageBytes = G * kABytes + kBBytes;
+  constexpr uint32_t kTmemCols = 2 * G * BN;  // two sets of G accumulators
   constexpr uint32_t kIdesc = make_idesc(BN, BF16);
+  // consumers of a queue entry: gather warps, W loader, MMA thread, epilogue warps
+  constexpr uint32_t kQueueReaders = kWarpsPerSlot * STAGES + 1 + 1 + 4;
+  static_assert(kTmemCols >= 32 && kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0,
+                "tensor memory columns");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * kStageBytes);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 1);
+  // barriers: full[S], empty[S], tfull[2], tempty[2], qfull[Q], qempty[Q]
+  Group<G>* queue = reinterpret_cast<Group<G>*>(bars + 2 * STAGES + 4 + 2 * kQueue);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(queue + kQueue);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int tile = args.n_tiles - 1 - int(blockIdx.x);  // largest tap sets first
-  const int n0 = int(blockIdx.y) * BN;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kb_per_tap = args.cin / kBK;
-  int slot0 = 0, ntaps = 1;
-  if (!args.dense) {
-    slot0 = args.tile_off[tile];
-    ntaps = args.tile_off[tile + 1] - slot0;
-  }
-  const int iters = ntaps * kb_per_tap;
+  const int total_work = args.n_groups * args.n_blocks;
   const uint32_t full0 = smem_addr(bars);
   const uint32_t empty0 = smem_addr(bars + STAGES);
-  const uint32_t accum_bar = smem_addr(bars + 2 * STAGES);
+  const uint32_t tfull0 = smem_addr(bars + 2 * STAGES);
+  const uint32_t tempty0 = smem_addr(bars + 2 * STAGES + 2);
+  const uint32_t qfull0 = smem_addr(bars + 2 * STAGES + 4);
+  const uint32_t qempty0 = smem_addr(bars + 2 * STAGES + 4 + kQueue);
 
-  if (tid == 0) {
+  if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full0 + 8 * s, 4 * 32 + 1);
+      mbar_init(full0 + 8 * s, kWarpsPerSlot * 32 + 1);  // gather lanes + the W loader
       mbar_init(empty0 + 8 * s, 1);
     }
-    mbar_init(accum_bar, 1);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull0 + 8 * a, 1);
+      mbar_init(tempty0 + 8 * a, 4 * 32);
+    }
+    for (int q = 0; q < kQueue; ++q) {
+      mbar_init(qfull0 + 8 * q, 1);
+      mbar_init(qempty0 + 8 * q, kQueueReaders);
+    }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 5) tmem_alloc(smem_addr(tmem_slot), kTmemCols);
+  if (warp == 1) tmem_alloc(smem_addr(tmem_slot), kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp < 4) {
-    // ---------------- gather producer ----------------
-    const int chunk = tid & 7;  // 16-byte chunk of a row's 128-byte slice
-    const int rsub = tid >> 3;  // rows rsub + 16 j, j = 0..7
-    int g[8];
-    int issued = 0;
-    for (int it = 0; it < iters; ++it) {
-      const int s = it / kb_per_tap;
-      const int kb = it - s * kb_per_tap;
-      if (kb == 0) {
+  // Next work item from the queue; every unit (a warp, or one thread) reads
+  // each entry once and releases it with one arrival.  warp_wide: all 32
+  // lanes read and lane 0 releases after the warp has read.  Returns w = -1
+  // at the end or when the CTA aborts.
+  auto next_item = [&](uint32_t& j, bool warp_wide) -> Group<G> {
+    Group<G> gr;
+    const uint32_t q = j % kQueue;
+    bool ok = mbar_wait(qfull0 + 8 * q, (j / kQueue) & 1, abort_flag, args.status);
+    if (warp_wide) ok = __all_sync(0xffffffffu, ok);
+    if (!ok) {
+      gr.w = -1;
+      return gr;
+    }
+    gr = queue[q];
+    if (warp_wide) __syncwarp();
+    if (!warp_wide || lane == 0) mbar_arrive(qempty0 + 8 * q);
+    ++j;
+    return gr;
+  };
+
+  if (warp == kPrefetchWarp) {
+    // ---------------- scheduler: hands out items ----------------
+    for (uint32_t j = 0;; ++j) {
+      const uint32_t q = j % kQueue;
+      int w = -1;
+      if (lane == 0) {
+        if (mbar_wait(qempty0 + 8 * q, ((j / kQueue) & 1) ^ 1, abort_flag, args.status)) {
+          const uint32_t t = atomicAdd(args.work_counter, 1u);
+          w = t < uint32_t(total_work) ? int(t) : -1;
+        }
+      }
+      w = __shfl_sync(0xffffffffu, w, 0);
+      Group<G> gr;
+      if (w >= 0) {
+        gr = group_of<BN, G>(args, w);
+      } else {
+        gr.w = -1;
+      }
+      if (lane == 0) {
+        queue[q] = gr;
+        mbar_arrive(qfull0 + 8 * q);  // release: publishes the entry
+      }
+      if (w < 0) break;
+    }
+  } else if (warp >= kFirstGatherWarp) {
+    // ---------------- gather warps: warps 4 i .. 4 i + 3 own stage slot i ----
+    const int gw = (warp - kFirstGatherWarp) / kWarpsPerSlot;  // slot
+    const int rq = (warp - kFirstGatherWarp) % kWarpsPerSlot;  // rows 32 rq .. 32 rq + 31
+    const int chunk = lane & 7;  // 16-byte chunk within a 128-byte row slice
+    const int rsub = lane >> 3;  // instruction j copies local rows 4 j + rsub
+    // The index loads of an owned stage are issued one owned stage ahead of
+    // its copies, so they overlap the wait for the slot.
+    GatherJob<G> pend;
+    bool have_pend = false;
+    bool ok = true;
+    auto run = [&](const GatherJob<G>& job) -> bool {
+      if (!mbar_wait(empty0 + 8 * job.stage, ((job.g / STAGES) & 1) ^ 1, abort_flag,
+                     args.status))
+        return false;
+      const uint32_t stage_base = smem_addr(smem + job.stage * kStageBytes);
+      const uint16_t* src_col = args.feats + job.kb * kBK + chunk * 8;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int row = rsub + 16 * j;
-          if (args.dense) {
-            const int64_t r = int64_t(tile) * kTileRows + row;
-            g[j] = r < args.n ? int(r) : -1;
-          } else {
-            g[j] = args.gidx[int64_t(slot0 + s) * kTileRows + row];
+      for (int k = 0; k < G; ++k) {
+        if (!((job.tiles >> k) & 1u)) continue;
+        const uint32_t a_base = stage_base + k * kABytes;
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const int local = 4 * jj + rsub;
+          const int v = __shfl_sync(0xffffffffu, job.vidx[k], local);
+          const int row = 32 * rq + local;
+          const uint16_t* src = v >= 0 ? src_col + int64_t(v) * args.cin : args.feats;
+          cp_async_16(a_base + row * 128 + ((chunk ^ (row & 7)) << 4), src, v >= 0 ? 16u : 0u);
+        }
+      }
+      cp_async_arrive_noinc(full0 + 8 * job.stage);
+      return true;
+    };
+    uint32_t g = 0, j = 0;
+    while (ok) {
+      const Group<G> cur = next_item(j, true);
+      if (cur.w < 0) break;
+      uint32_t rem = rotate_taps(cur.all, cur.rot);
+      while (rem && ok) {
+        const int tap = next_tap(rem, cur.rot);
+        for (int kb = 0; kb < kb_per_tap && ok; ++kb, ++g) {
+          const int stage = int(g % STAGES);
+          if (stage != gw) continue;
+          GatherJob<G> job;
+          job.stage = stage;
+          job.g = g;
+          job.kb = kb;
+          job.tiles = 0;
+#pragma unroll
+          for (int k = 0; k < G; ++k) {
+            job.vidx[k] = -1;
+            if (!((cur.mask[k] >> tap) & 1u)) continue;
+            job.tiles |= 1u << k;
+            if (args.dense) {
+              const int64_t r = int64_t(cur.tile0 + k) * kTileRows + 32 * rq + lane;
+              job.vidx[k] = r < args.n ? int(r) : -1;
+            } else {
+              const int slot = cur.slot0[k] + __popc(cur.mask[k] & ((1u << tap) - 1u));
+              job.vidx[k] = args.gidx[int64_t(slot) * kTileRows + 32 * rq + lane];
+            }
+          }
+          if (have_pend) ok = run(pend);
+          pend = job;
+          have_pend = true;
+        }
+      }
+    }
+    if (have_pend && ok) run(pend);
+    asm volatile("cp.async.wait_all;" ::: "memory");
+  } else if (warp == 0) {
+    // ---------------- W loader ----------------
+    if (lane == 0) {
+      tma_prefetch_map(&wmap);
+      uint32_t g = 0, j = 0;
+      bool ok = true;
+      while (ok) {
+        const Group<G> cur = next_item(j, false);
+        if (cur.w < 0) break;
+        uint32_t rem = rotate_taps(cur.all, cur.rot);
+        while (rem && ok) {
+          const int tap = next_tap(rem, cur.rot);
+          for (int kb = 0; kb < kb_per_tap; ++kb, ++g) {
+            const int stage = int(g % STAGES);
+            if (!mbar_wait(empty0 + 8 * stage, ((g / STAGES) & 1) ^ 1, abort_flag, args.status)) {
+              ok = false;
+              break;
+            }
+            const uint32_t full = full0 + 8 * stage;
+            mbar_arrive_expect_tx(full, kBBytes);
+            const uint32_t b_base = smem_addr(smem + stage * kStageBytes + G * kABytes);
+#pragma unroll
+            for (int jj = 0; jj < BN / 64; ++jj)
+              tma_load_2d(b_base + jj * (kBK * 128), &wmap, cur.n0 + 64 * jj,
+                          tap * args.cin + kb * kBK, full);
           }
         }
       }
-      const int stage = it % STAGES;
-      if (!mbar_wait(empty0 + 8 * stage, ((it / STAGES) & 1) ^ 1, abort_flag, args.status)) break;
-      const uint32_t a_base = smem_addr(smem + stage * kStageBytes);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int row = rsub + 16 * j;
-        const bool ok = g[j] >= 0;
-        const uint16_t* src =
-            ok ? args.feats + int64_t(g[j]) * args.cin + kb * kBK + chunk * 8 : args.feats;
-        cp_async_16(a_base + row * 128 + ((chunk ^ (row & 7)) << 4), src, ok ? 16u : 0u);
-      }
-      cp_async_commit();
-      ++issued;
-      if (it >= LAG) {
-        cp_async_wait<LAG>();
-        fence_async_proxy();
-        mbar_arrive(full0 + 8 * ((it - LAG) % STAGES));
-      }
     }
-    cp_async_wait<0>();
-    fence_async_proxy();
-    for (int it = issued > LAG ? issued - LAG : 0; it < issued; ++it)
-      mbar_arrive(full0 + 8 * (it % STAGES));
-
-    // ---------------- epilogue ----------------
-    bool have = iters > 0 && mbar_wait(accum_bar, 0, abort_flag, args.status);
-    have = __all_sync(0xffffffffu, have);  // tcgen05.ld below is warp-collective
-    tc_fence_after();
-    const int row = warp * 32 + lane;
-    int32_t orow;
-    if (args.dense) {
-      const int64_t r = int64_t(tile) * kTileRows + row;
-      orow = r < args.n ? int32_t(r) : -1;
-    } else {
-      orow = args.out_row[int64_t(tile) * kTileRows + row];
-    }
-    uint16_t* dst = args.out + int64_t(orow < 0 ? 0 : orow) * args.cout + n0;
-#pragma unroll 1
-    for (int cc = 0; cc < BN / 32; ++cc) {
-      uint32_t v[32];
-      if (have) {
-        tmem_ld_x32(tmem + (uint32_t(warp * 32) << 16) + uint32_t(cc * 32), v);
-      } else {
-#pragma unroll
-        for (int q = 0; q < 32; ++q) v[q] = 0u;
-      }
-      if (orow >= 0 && !*abort_flag) {
-        uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint4 w;
-          w.x = pack2<BF16>(v[8 * q + 0], v[8 * q + 1]);
-          w.y = pack2<BF16>(v[8 * q + 2], v[8 * q + 3]);
-          w.z = pack2<BF16>(v[8 * q + 4], v[8 * q + 5]);
-          w.w = pack2<BF16>(v[8 * q + 6], v[8 * q + 7]);
-          d4[q] = w;
-        }
-      }
-    }
-  } else if (warp == 4) {
-    // ---------------- W producer (TMA) ----------------
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      tma_prefetch_map(&wmap);
-      for (int it = 0; it < iters; ++it) {
-        const int s = it / kb_per_tap;
-        const int kb = it - s * kb_per_tap;
-        const int tap = args.dense ? 0 : int(args.tile_taps[int64_t(tile) * 32 + s]);
-        const int stage = it % STAGES;
-        if (!mbar_wait(empty0 + 8 * stage, ((it / STAGES) & 1) ^ 1, abort_flag, args.status))
+      uint32_t g = 0, j = 0, acc_iter = 0;
+      bool ok = true;
+      const uint64_t adesc0 = desc_a_kmajor(smem_addr(smem));
+      const uint64_t bdesc0 = desc_b_mnmajor(smem_addr(smem) + G * kABytes, kBK * 128);
+      while (ok) {
+        const Group<G> cur = next_item(j, false);
+        if (cur.w < 0) break;
+        const uint32_t a = acc_iter & 1;
+        if (!mbar_wait(tempty0 + 8 * a, ((acc_iter >> 1) & 1) ^ 1, abort_flag, args.status)) {
+          ok = false;
           break;
-        const uint32_t full = full0 + 8 * stage;
-        mbar_arrive_expect_tx(full, kBBytes);
-        const uint32_t b_base = smem_addr(smem + stage * kStageBytes + kABytes);
+        }
+        tc_fence_after();
+        uint32_t started = 0;  // bit k: tile k's accumulator holds a partial sum
+        uint32_t rem = rotate_taps(cur.all, cur.rot);
+        while (rem && ok) {
+          const int tap = next_tap(rem, cur.rot);
+          for (int kb = 0; kb < kb_per_tap; ++kb, ++g) {
+            const int stage = int(g % STAGES);
+            if (!mbar_wait(full0 + 8 * stage, (g / STAGES) & 1, abort_flag, args.status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            // descriptors of this stage: the start-address field (bits 0-13,
+            // 16-byte units) never carries, so offsets add to the 64-bit value
+            const uint64_t soff = uint64_t(stage) * (kStageBytes >> 4);
 #pragma unroll
-        for (int j = 0; j < BN / 64; ++j)
-          tma_load_2d(b_base + j * (kBK * 128), &wmap, n0 + 64 * j, tap * args.cin + kb * kBK,
-                      full);
+            for (int k = 0; k < G; ++k) {
+              if (!((cur.mask[k] >> tap) & 1u)) continue;
+              const uint32_t d_tmem = tmem + (a * G + k) * BN;
+              const uint64_t ad = adesc0 + soff + uint64_t(k * (kABytes >> 4));
+              const uint64_t bd = bdesc0 + soff;
+              const uint32_t acc = (started >> k) & 1u;
+#pragma unroll
+              for (int kk = 0; kk < kBK / 16; ++kk)
+                umma_f16(d_tmem, ad + 2 * kk, bd + (2048 >> 4) * kk, kIdesc, kk != 0 ? 1u : acc);
+              started |= 1u << k;
+            }
+            umma_commit(empty0 + 8 * stage);
+          }
+        }
+        umma_commit(tfull0 + 8 * a);
+        if (!ok) mbar_drain(tfull0 + 8 * a, (acc_iter >> 1) & 1);
+        ++acc_iter;
       }
     }
     __syncwarp();
   } else {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
-      int done = 0;
-      for (int it = 0; it < iters; ++it) {
-        const int stage = it % STAGES;
-        if (!mbar_wait(full0 + 8 * stage, (it / STAGES) & 1, abort_flag, args.status)) break;
-        tc_fence_after();
-        const uint32_t a_base = smem_addr(smem + stage * kStageBytes);
-        const uint32_t b_base = a_base + kABytes;
+    // ---------------- epilogue (warps 2-5) ----------------
+    const int quarter = warp & 3;  // tensor-memory lanes 32*quarter .. +31
+    const int row = quarter * 32 + lane;
+    uint32_t j = 0, acc_iter = 0;
+    while (true) {
+      const Group<G> gr = next_item(j, true);
+      if (gr.w < 0) break;
+      int32_t orow[G];
 #pragma unroll
-        for (int k = 0; k < kBK / 16; ++k) {
-          umma_f16(tmem, desc_a_kmajor(a_base + 32 * k), desc_b_mnmajor(b_base + 2048 * k, kBK * 128),
-                   kIdesc, (it | k) != 0 ? 1u : 0u);
+      for (int k = 0; k < G; ++k) {
+        const int64_t r = int64_t(gr.tile0 + k) * kTileRows + row;
+        if (gr.mask[k] == 0)
+          orow[k] = -1;
+        else if (args.dense)
+          orow[k] = r < args.n ? int32_t(r) : -1;
+        else
+          orow[k] = args.out_row[r];
+      }
+      const uint32_t a = acc_iter & 1;
+      bool have = mbar_wait(tfull0 + 8 * a, (acc_iter >> 1) & 1, abort_flag, args.status);
+      have = __all_sync(0xffffffffu, have);  // tcgen05.ld below is warp-collective
+      if (!have) break;
+      tc_fence_after();
+#pragma unroll
+      for (int k = 0; k < G; ++k) {
+        if (gr.mask[k] == 0) continue;  // past the last tile
+        uint16_t* dst = args.out + int64_t(orow[k] < 0 ? 0 : orow[k]) * args.cout + gr.n0;
+#pragma unroll 1
+        for (int cc = 0; cc < BN / 32; ++cc) {
+          uint32_t v[32];
+          tmem_ld_x32(tmem + (uint32_t(quarter * 32) << 16) + (a * G + k) * BN + uint32_t(cc * 32),
+                      v);
+          if (orow[k] >= 0) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint4 o;
+              o.x = pack2<BF16>(v[8 * q + 0], v[8 * q + 1]);
+              o.y = pack2<BF16>(v[8 * q + 2], v[8 * q + 3]);
+              o.z = pack2<BF16>(v[8 * q + 4], v[8 * q + 5]);
+              o.w = pack2<BF16>(v[8 * q + 6], v[8 * q + 7]);
+              d4[q] = o;
+            }
+          }
         }
-        umma_commit(empty0 + 8 * stage);
-        ++done;
       }
-      umma_commit(accum_bar);
-      if (done < iters) {
-        // aborted: let the MMAs already issued finish before the memory goes away
-        mbar_drain(accum_bar, 0);
-      }
+      tc_fence_before();
+      mbar_arrive(tempty0 + 8 * a);
+      ++acc_iter;
     }
-    __syncwarp();
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -410,12 +617,37 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   return fn;
 }
 
-template <int BN, int STAGES, int LAG, bool BF16>
+int sm_count() {
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+    sms = 148;
+  return sms;
+}
+
+// 2-D row-major [rows][cols] tensor map with a (64 x box_rows) box and
+// 128-byte swizzle.
+bool encode_2d(CUtensorMap* map, bool bf16, const void* base, uint64_t cols, uint64_t rows,
+               uint32_t box_rows) {
+  auto encode = get_encode_fn();
+  if (!encode) return false;
+  cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(cols) * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return encode(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, int STAGES, int G, bool BF16>
 int launch_cfg(const Plan& plan, bool dense, const void* feats, const void* W, void* out, int cin,
                int cout, cudaStream_t stream) {
-  constexpr int kStageBytes = kABytes + BN * kBK * 2;
-  constexpr int kSmem = STAGES * kStageBytes + 1024 + 256;
-  auto kern = k_conv_tc<BN, STAGES, LAG, BF16>;
+  constexpr int kStageBytes = G * kABytes + BN * kBK * 2;
+  constexpr int kSmem = STAGES * kStageBytes + 1024 + 512;
+  static_assert(kSmem <= 227 * 1024, "shared memory");
+  auto kern = k_conv_tc<BN, STAGES, G, BF16>;
   static bool attr_set = false;
   if (!attr_set) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) !=
@@ -423,43 +655,57 @@ int launch_cfg(const Plan& plan, bool dense, const void* feats, const void* W, v
       return SMC_ERR_CUDA;
     attr_set = true;
   }
-  auto encode = get_encode_fn();
-  if (!encode) return SMC_ERR_CUDA;
+  CUtensorMap wmap;
   const int taps = dense ? 1 : kTaps;
-  CUtensorMap map;
-  cuuint64_t dims[2] = {cuuint64_t(cout), cuuint64_t(taps) * cuuint64_t(cin)};
-  cuuint64_t strides[1] = {cuuint64_t(cout) * 2};
-  cuuint32_t box[2] = {64, kBK};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = encode(&map, BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-                      2, const_cast<void*>(W), dims, strides, box, estr,
-                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return SMC_ERR_CUDA;
+  if (!encode_2d(&wmap, BF16, W, uint64_t(cout), uint64_t(taps) * uint64_t(cin), kBK))
+    return SMC_ERR_CUDA;
   ConvArgs a;
   a.feats = static_cast<const uint16_t*>(feats);
   a.out = static_cast<uint16_t*>(out);
   a.gidx = plan.gidx;
   a.tile_off = plan.tile_off;
-  a.tile_taps = plan.tile_taps;
+  a.tile_mask = plan.tile_mask;
   a.out_row = plan.out_row;
   a.status = plan.status;
   a.n = plan.n;
   a.cin = cin;
   a.cout = cout;
   a.n_tiles = int(plan.n_tiles);
+  a.n_blocks = cout / BN;
+  a.n_groups = int((plan.n_tiles + G - 1) / G);
   a.dense = dense ? 1 : 0;
-  dim3 grid(unsigned(plan.n_tiles), unsigned(cout / BN));
-  kern<<<grid, kThreads, kSmem, stream>>>(map, a);
+  a.work_counter = plan.work_counter;
+  if (cudaMemsetAsync(plan.work_counter, 0, sizeof(uint32_t), stream) != cudaSuccess)
+    return SMC_ERR_CUDA;
+  const int64_t work = int64_t(a.n_groups) * a.n_blocks;
+  const int grid = int(std::min<int64_t>(work, sm_count()));
+  kern<<<grid, threads_for(STAGES), kSmem, stream>>>(wmap, a);
   return cudaGetLastError() == cudaSuccess ? SMC_OK : SMC_ERR_CUDA;
+}
+
+// Tile-group size override for tuning (SMC_TC_GROUP=1 or 2; default 2 for
+// BN < 256), read once.
+int group_override() {
+  static int v = [] {
+    const char* e = std::getenv("SMC_TC_GROUP");
+    return e ? std::atoi(e) : 0;
+  }();
+  return v;
 }
 
 template <bool BF16>
 int launch_dtype(const Plan& plan, bool dense, const void* feats, const void* W, void* out,
                  int cin, int cout, cudaStream_t stream) {
-  if (cout % 256 == 0) return launch_cfg<256, 4, 2, BF16>(plan, dense, feats, W, out, cin, cout, stream);
-  if (cout % 128 == 0) return launch_cfg<128, 3, 1, BF16>(plan, dense, feats, W, out, cin, cout, stream);
-  return launch_cfg<64, 4, 2, BF16>(plan, dense, feats, W, out, cin, cout, stream);
+  if (group_override() == 1 && cout % 256 != 0) {
+    if (cout % 128 == 0)
+      return launch_cfg<128, 5, 1, BF16>(plan, dense, feats, W, out, cin, cout, stream);
+    return launch_cfg<64, 6, 1, BF16>(plan, dense, feats, W, out, cin, cout, stream);
+  }
+  if (cout % 256 == 0)
+    return launch_cfg<256, 4, 1, BF16>(plan, dense, feats, W, out, cin, cout, stream);
+  if (cout % 128 == 0)
+    return launch_cfg<128, 4, 2, BF16>(plan, dense, feats, W, out, cin, cout, stream);
+  return launch_cfg<64, 5, 2, BF16>(plan, dense, feats, W, out, cin, cout, stream);
 }
 
 }  // namespace

@@ -329,6 +329,7 @@ int build_plan_impl(const int32_t* coords, int64_t n, int32_t stride, int64_t ta
                     int32_t order, cudaStream_t s, Plan* plan, Scratch& sc) {
   const int4* c4 = reinterpret_cast<const int4*>(coords);
   SMC_TRY(dev_alloc(&plan->status, 1, s));
+  SMC_TRY(dev_alloc(&plan->work_counter, 64, s));
   if (cudaMemsetAsync(plan->status, 0, sizeof(int32_t), s) != cudaSuccess) return SMC_ERR_CUDA;
   plan->n = n;
   plan->n_tiles = (n + kTileRows - 1) / kTileRows;
@@ -445,6 +446,7 @@ void free_plan(Plan* plan) {
   dev_free(plan->gidx, s);
   dev_free(plan->out_row, s);
   dev_free(plan->status, s);
+  dev_free(plan->work_counter, s);
   cudaStreamSynchronize(s);
 }
 
