@@ -288,7 +288,8 @@ struct GatherJob {
   int vidx[G];     // lane l: source row of local row l of tile k (-1 = zero row)
 };
 
-constexpr int kQueue = 4;  // work items published ahead of the consumers
+constexpr int kQueue = 2;  // work items published ahead of the producers (small: a
+                           // reserved item cannot move to an idle SM)
 
 template <int BN, int STAGES, int G, bool BF16>
 __global__ void __launch_bounds__(threads_for(STAGES), 1)
@@ -298,8 +299,9 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const ConvArgs args) {
   constexpr int kStageBytes = G * kABytes + kBBytes;
   constexpr uint32_t kTmemCols = 2 * G * BN;  // two sets of G accumulators
   constexpr uint32_t kIdesc = make_idesc(BN, BF16);
-  // consumers of a queue entry: gather warps, W loader, MMA thread, epilogue warps
-  constexpr uint32_t kQueueReaders = kWarpsPerSlot * STAGES + 1 + 1 + 4;
+  // readers of a queue entry: gather warps, W loader, MMA thread (the epilogue
+  // learns each item from the MMA thread, one accumulator at a time)
+  constexpr uint32_t kQueueReaders = kWarpsPerSlot * STAGES + 1 + 1;
   static_assert(kTmemCols >= 32 && kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0,
                 "tensor memory columns");
 
@@ -307,9 +309,10 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const ConvArgs args) {
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * kStageBytes);
-  // barriers: full[S], empty[S], tfull[2], tempty[2], qfull[Q], qempty[Q]
-  Group<G>* queue = reinterpret_cast<Group<G>*>(bars + 2 * STAGES + 4 + 2 * kQueue);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(queue + kQueue);
+  // barriers: full[S], empty[S], tfull[2], tempty[2], qfull[Q], qempty[Q], info[2]
+  Group<G>* queue = reinterpret_cast<Group<G>*>(bars + 2 * STAGES + 6 + 2 * kQueue);
+  Group<G>* acc_info = queue + kQueue;  // item held by each accumulator
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_info + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -321,6 +324,7 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const ConvArgs args) {
   const uint32_t tempty0 = smem_addr(bars + 2 * STAGES + 2);
   const uint32_t qfull0 = smem_addr(bars + 2 * STAGES + 4);
   const uint32_t qempty0 = smem_addr(bars + 2 * STAGES + 4 + kQueue);
+  const uint32_t info0 = smem_addr(bars + 2 * STAGES + 4 + 2 * kQueue);  // 2 barriers
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -330,6 +334,7 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const ConvArgs args) {
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull0 + 8 * a, 1);
       mbar_init(tempty0 + 8 * a, 4 * 32);
+      mbar_init(info0 + 8 * a, 1);
     }
     for (int q = 0; q < kQueue; ++q) {
       mbar_init(qfull0 + 8 * q, 1);
@@ -394,8 +399,8 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const ConvArgs args) {
     const int rq = (warp - kFirstGatherWarp) % kWarpsPerSlot;  // rows 32 rq .. 32 rq + 31
     const int chunk = lane & 7;  // 16-byte chunk within a 128-byte row slice
     const int rsub = lane >> 3;  // instruction j copies local rows 4 j + rsub
-    // The index loads of an owned stage are issued one owned stage ahead of
-    // its copies, so they overlap the wait for the slot.
+    // Within an item, the index loads of an owned stage are issued one owned
+    // stage ahead of its copies, so they overlap the wait for the slot.
     GatherJob<G> pend;
     bool have_pend = false;
     bool ok = true;
@@ -454,8 +459,12 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const ConvArgs args) {
           have_pend = true;
         }
       }
+      // Never carry a stage into the next item: the next owned stage may lie
+      // several items ahead, which the queue only publishes once the MMA
+      // thread has moved on -- and the MMA thread waits for this stage.
+      if (have_pend && ok) ok = run(pend);
+      have_pend = false;
     }
-    if (have_pend && ok) run(pend);
     asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == 0) {
     // ---------------- W loader ----------------
@@ -496,12 +505,16 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const ConvArgs args) {
       const uint64_t bdesc0 = desc_b_mnmajor(smem_addr(smem) + G * kABytes, kBK * 128);
       while (ok) {
         const Group<G> cur = next_item(j, false);
-        if (cur.w < 0) break;
         const uint32_t a = acc_iter & 1;
         if (!mbar_wait(tempty0 + 8 * a, ((acc_iter >> 1) & 1) ^ 1, abort_flag, args.status)) {
           ok = false;
           break;
         }
+        // tell the epilogue which item this accumulator will hold (or that
+        // there are no more); the buffer's epilogue has finished with it
+        acc_info[a] = cur;
+        mbar_arrive(info0 + 8 * a);
+        if (cur.w < 0) break;
         tc_fence_after();
         uint32_t started = 0;  // bit k: tile k's accumulator holds a partial sum
         uint32_t rem = rotate_taps(cur.all, cur.rot);
@@ -542,9 +555,13 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const ConvArgs args) {
     // ---------------- epilogue (warps 2-5) ----------------
     const int quarter = warp & 3;  // tensor-memory lanes 32*quarter .. +31
     const int row = quarter * 32 + lane;
-    uint32_t j = 0, acc_iter = 0;
+    uint32_t acc_iter = 0;
     while (true) {
-      const Group<G> gr = next_item(j, true);
+      const uint32_t a = acc_iter & 1;
+      bool have = mbar_wait(info0 + 8 * a, (acc_iter >> 1) & 1, abort_flag, args.status);
+      have = __all_sync(0xffffffffu, have);
+      if (!have) break;
+      const Group<G> gr = acc_info[a];
       if (gr.w < 0) break;
       int32_t orow[G];
 #pragma unroll
@@ -557,8 +574,7 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const ConvArgs args) {
         else
           orow[k] = args.out_row[r];
       }
-      const uint32_t a = acc_iter & 1;
-      bool have = mbar_wait(tfull0 + 8 * a, (acc_iter >> 1) & 1, abort_flag, args.status);
+      have = mbar_wait(tfull0 + 8 * a, (acc_iter >> 1) & 1, abort_flag, args.status);
       have = __all_sync(0xffffffffu, have);  // tcgen05.ld below is warp-collective
       if (!have) break;
       tc_fence_after();

@@ -154,3 +154,53 @@ def test_workload_resblock64_pair_sampled():
     ref1, scale1 = native.submconv(h_cpu, inp.weights[1].double().numpy(), ident, rows=rows)
     check_conv(y[r_idx], ref1, scale1, "resblock 1x1x1")
     idx.close()
+
+
+@pytest.mark.parametrize("cout", [64, 128, 256])
+def test_many_single_stage_work_items(cout):
+    """Isolated voxels give one-tap tiles (one or two pipeline stages per work
+    item); the kernel must hand items to every role without waiting on later
+    items."""
+    pts = np.array([[b, 3 * i, 3 * j, 3 * k] for b in range(2) for i in range(12)
+                    for j in range(12) for k in range(12)], np.int32)
+    rng = np.random.default_rng(41 + cout)
+    feats = synth.round_to(rng.standard_normal((len(pts), 64)), "bf16")
+    W = synth.round_to(rng.standard_normal((27, 64, cout)) / 8.0, "bf16")
+    idx, out = _run(pts, feats, W, 3)
+    ref, scale = oracle_conv(pts, feats, W, 3)
+    check_conv(out, ref, scale, f"isolated cout={cout}")
+    idx.close()
+
+
+_GROUP1_SCRIPT = r"""
+import sys, numpy as np, torch
+sys.path.insert(0, {root!r}); sys.path.insert(0, {tests!r})
+from submanifold_sparse_convolution_coord_b200 import synth
+from submanifold_sparse_convolution_coord_b200.binding import SubMIndex
+from gpu_common import check_conv, oracle_conv
+cases = [(0, 3000, 20, 1, 128, 128, "f16"), (1, 800, 40, 2, 64, 64, "bf16"), (2, 2000, 16, 1, 64, 128, "f16")]
+for seed, n, grid, batch, cin, cout, dt in cases:
+    coords, feats, W = synth.random_case(seed, n, grid, batch, cin, cout, 3, dt, True)
+    idx = SubMIndex(torch.from_numpy(coords).cuda())
+    out = idx.forward(feats.cuda(), W.cuda())
+    torch.cuda.synchronize()
+    assert idx.status() == 0
+    ref, scale = oracle_conv(coords, feats, W, 3)
+    check_conv(out, ref, scale, str((seed, cin, cout)))
+    idx.close()
+print("ok")
+"""
+
+
+def test_group_size_one_configuration():
+    """The tile-group-size override (one tile per work item) in a fresh
+    process, since the setting is read once per process."""
+    import os
+    import subprocess
+    import sys
+    here = os.path.dirname(os.path.abspath(__file__))
+    code = _GROUP1_SCRIPT.format(root=os.path.dirname(here), tests=here)
+    env = dict(os.environ, SMC_TC_GROUP="1")
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0 and "ok" in r.stdout, r.stdout + r.stderr
