@@ -135,8 +135,12 @@ int smc_build_neighbor_map_static(const int32_t* coords_dev, int64_t n, int32_t 
  *         atomics; every element is overwritten.
  * K     : 3 (uses the neighbour map) or 1 (per-row linear map, ignores it).
  * dtype : SMC_F16 / SMC_BF16 -- tensor cores, fp32 accumulation, output
- *         rounded to nearest; SMC_F32 -- fp32 FMA on the CUDA cores.
+ *         rounded to nearest; SMC_F32 -- CUDA cores, fp64 accumulation,
+ *         output rounded once to fp32.
  * stream: the call is asynchronous on this stream and never synchronises.
+ *         Forward calls that use the same handle must be ordered (one stream,
+ *         or events): the tensor-core kernel keeps its work counter in the
+ *         handle.
  *
  * Tensor-core path when cin % 64 == 0 and cout % 64 == 0 (f16/bf16); any
  * other cin, cout >= 1 runs on the CUDA-core kernel.  feats and out must not
