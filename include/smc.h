@@ -56,7 +56,8 @@ enum smc_dtype { SMC_F32 = 0, SMC_F16 = 1, SMC_BF16 = 2 };
 
 /* Row order used for the tile plan (smc_index_options.order). */
 enum smc_order {
-  SMC_ORDER_MASK = 0,  /* rows sorted by (number of active taps, tap mask): default */
+  SMC_ORDER_MASK = 0,  /* rows sorted by (number of active taps, Gray-code rank of the
+                          tap mask): default */
   SMC_ORDER_INPUT = 1  /* rows in input order (ablation) */
 };
 

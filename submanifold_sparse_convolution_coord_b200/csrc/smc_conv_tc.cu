@@ -12,7 +12,8 @@
 //
 // Persistent kernel, one CTA per SM, 7 + 4 * STAGES warps:
 //   warp 0      lane 0 loads the W[tap] slice of each stage with TMA
-//               (MN-major, 128-byte swizzle);
+//               (MN-major, 128-byte swizzle), and for K = 1 also the stage's
+//               contiguous feature rows (128 x 64 box, 128-byte swizzle);
 //   warp 1      allocates tensor memory; lane 0 issues the MMAs (M = 128,
 //               N = BN, K = 16) into one of two accumulators;
 //   warps 2-5   epilogue: tensor memory -> registers -> fp16/bf16 -> global,
@@ -293,7 +294,8 @@ constexpr int kQueue = 2;  // work items published ahead of the producers (small
 
 template <int BN, int STAGES, int G, bool BF16>
 __global__ void __launch_bounds__(threads_for(STAGES), 1)
-k_conv_tc(const __grid_constant__ CUtensorMap wmap, const ConvArgs args) {
+k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap fmap,
+          const ConvArgs args) {
   static_assert(BN % 64 == 0 && BN <= 256, "BN");
   constexpr int kBBytes = BN * kBK * 2;
   constexpr int kStageBytes = G * kABytes + kBBytes;
@@ -328,7 +330,9 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const ConvArgs args) {
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full0 + 8 * s, kWarpsPerSlot * 32 + 1);  // gather lanes + the W loader
+      // sparse: the gather lanes and the W loader; dense (K = 1): the loader
+      // brings the contiguous A rows with TMA too
+      mbar_init(full0 + 8 * s, args.dense ? 1 : kWarpsPerSlot * 32 + 1);
       mbar_init(empty0 + 8 * s, 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -430,6 +434,7 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const ConvArgs args) {
     while (ok) {
       const Group<G> cur = next_item(j, true);
       if (cur.w < 0) break;
+      if (args.dense) continue;  // the loader brings contiguous rows by TMA
       uint32_t rem = rotate_taps(cur.all, cur.rot);
       while (rem && ok) {
         const int tap = next_tap(rem, cur.rot);
@@ -446,13 +451,8 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const ConvArgs args) {
             job.vidx[k] = -1;
             if (!((cur.mask[k] >> tap) & 1u)) continue;
             job.tiles |= 1u << k;
-            if (args.dense) {
-              const int64_t r = int64_t(cur.tile0 + k) * kTileRows + 32 * rq + lane;
-              job.vidx[k] = r < args.n ? int(r) : -1;
-            } else {
-              const int slot = cur.slot0[k] + __popc(cur.mask[k] & ((1u << tap) - 1u));
-              job.vidx[k] = args.gidx[int64_t(slot) * kTileRows + 32 * rq + lane];
-            }
+            const int slot = cur.slot0[k] + __popc(cur.mask[k] & ((1u << tap) - 1u));
+            job.vidx[k] = args.gidx[int64_t(slot) * kTileRows + 32 * rq + lane];
           }
           if (have_pend) ok = run(pend);
           pend = job;
@@ -470,6 +470,7 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const ConvArgs args) {
     // ---------------- W loader ----------------
     if (lane == 0) {
       tma_prefetch_map(&wmap);
+      if (args.dense) tma_prefetch_map(&fmap);
       uint32_t g = 0, j = 0;
       bool ok = true;
       while (ok) {
@@ -485,8 +486,21 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const ConvArgs args) {
               break;
             }
             const uint32_t full = full0 + 8 * stage;
-            mbar_arrive_expect_tx(full, kBBytes);
-            const uint32_t b_base = smem_addr(smem + stage * kStageBytes + G * kABytes);
+            const uint32_t stage_base = smem_addr(smem + stage * kStageBytes);
+            if (args.dense) {
+              uint32_t live = 0;
+#pragma unroll
+              for (int k = 0; k < G; ++k) live += cur.mask[k] != 0u ? 1u : 0u;
+              mbar_arrive_expect_tx(full, kBBytes + live * kABytes);
+#pragma unroll
+              for (int k = 0; k < G; ++k)
+                if (cur.mask[k] != 0u)
+                  tma_load_2d(stage_base + k * kABytes, &fmap, kb * kBK,
+                              (cur.tile0 + k) * kTileRows, full);
+            } else {
+              mbar_arrive_expect_tx(full, kBBytes);
+            }
+            const uint32_t b_base = stage_base + G * kABytes;
 #pragma unroll
             for (int jj = 0; jj < BN / 64; ++jj)
               tma_load_2d(b_base + jj * (kBK * 128), &wmap, cur.n0 + 64 * jj,
@@ -671,9 +685,10 @@ int launch_cfg(const Plan& plan, bool dense, const void* feats, const void* W, v
       return SMC_ERR_CUDA;
     attr_set = true;
   }
-  CUtensorMap wmap;
+  CUtensorMap wmap, fmap;
   const int taps = dense ? 1 : kTaps;
-  if (!encode_2d(&wmap, BF16, W, uint64_t(cout), uint64_t(taps) * uint64_t(cin), kBK))
+  if (!encode_2d(&wmap, BF16, W, uint64_t(cout), uint64_t(taps) * uint64_t(cin), kBK) ||
+      !encode_2d(&fmap, BF16, feats, uint64_t(cin), uint64_t(plan.n), kTileRows))
     return SMC_ERR_CUDA;
   ConvArgs a;
   a.feats = static_cast<const uint16_t*>(feats);
@@ -695,7 +710,7 @@ int launch_cfg(const Plan& plan, bool dense, const void* feats, const void* W, v
     return SMC_ERR_CUDA;
   const int64_t work = int64_t(a.n_groups) * a.n_blocks;
   const int grid = int(std::min<int64_t>(work, sm_count()));
-  kern<<<grid, threads_for(STAGES), kSmem, stream>>>(wmap, a);
+  kern<<<grid, threads_for(STAGES), kSmem, stream>>>(wmap, fmap, a);
   return cudaGetLastError() == cudaSuccess ? SMC_OK : SMC_ERR_CUDA;
 }
 

@@ -8,8 +8,9 @@
 //               an open-addressing table (linear probing, SplitMix64 mixer);
 //   2. query    the 27 neighbours c + stride*d of every voxel -> int32 map
 //               [n][27] (-1 = absent) and a 27-bit tap mask per voxel;
-//   3. order    rows by (popcount(mask), mask) with a stable LSD radix sort,
-//               so a 128-row tile holds voxels whose active taps coincide;
+//   3. order    rows by (popcount(mask), Gray-code rank of mask) with a stable
+//               LSD radix sort, so a 128-row tile holds voxels whose active
+//               taps coincide;
 //   4. plan     per tile, the OR of its rows' masks (the taps the tensor-core
 //               kernel multiplies; the others are skipped) and a compact
 //               gather index [tile][active tap][128 rows].
@@ -110,13 +111,22 @@ k_neighbors(const int4* __restrict__ coords, int64_t n, int32_t stride,
   }
 }
 
-// Sort key: popcount in the top 5 bits, then the 27-bit mask.
+// Sort key: popcount in the top 5 bits (so tiles come out lightest to
+// heaviest), then the rank of the 27-bit mask in reflected Gray-code order
+// (the prefix XOR of the mask): consecutive masks in that order differ in one
+// tap, so a 128-row run covers fewer distinct taps than in plain binary order.
 __global__ void k_sort_keys(const uint32_t* __restrict__ mask, int64_t n, uint32_t* keys,
                             int32_t* vals) {
   const int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
   if (i >= n) return;
   const uint32_t m = mask[i];
-  keys[i] = (uint32_t(__popc(m)) << 27) | m;
+  uint32_t r = m;
+  r ^= r >> 1;
+  r ^= r >> 2;
+  r ^= r >> 4;
+  r ^= r >> 8;
+  r ^= r >> 16;
+  keys[i] = (uint32_t(__popc(m)) << 27) | r;
   vals[i] = int32_t(i);
 }
 
