@@ -49,12 +49,10 @@ namespace {
 
 constexpr int kPrefetchWarp = 6;
 constexpr int kFirstGatherWarp = 7;
-constexpr int kWarpsPerSlot = 4;  // each copies 32 of a tile's 128 rows
-__host__ __device__ constexpr int threads_for(int stages) {
-  return 32 * (kFirstGatherWarp + kWarpsPerSlot * stages);
+// gather warps per stage slot (each copies 128 / WPS of a tile's rows)
+__host__ __device__ constexpr int threads_for(int stages, int wps) {
+  return 32 * (kFirstGatherWarp + wps * stages);
 }
-constexpr int kBK = 64;                          // input channels per stage (128 bytes)
-constexpr int kABytes = kTileRows * kBK * 2;     // 16 KB
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
 // ----------------------------------------------------------------------------
@@ -184,10 +182,15 @@ __device__ __forceinline__ void tmem_ld_x32(uint32_t taddr, uint32_t (&v)[32]) {
 // Shared-memory matrix descriptors (sm_100 UMMA format: start >> 4 in bits
 // 0-13, leading byte offset >> 4 in 16-29, stride byte offset >> 4 in 32-45,
 // version 1 in bit 46, layout type in 61-63 with 2 = 128-byte swizzle).
-// A: K-major, rows of 128 bytes, 8-row swizzle atoms 1024 bytes apart.
+// A: K-major, rows of 2*BK bytes (128 or 64) with the matching swizzle
+// (128-byte: layout 2, 64-byte: layout 4), 8-row atoms 16*BK bytes apart.
+template <int BK>
 __device__ __forceinline__ uint64_t desc_a_kmajor(uint32_t addr) {
-  return uint64_t((addr >> 4) & 0x3FFFu) | (uint64_t(1) << 16) | (uint64_t(1024 >> 4) << 32) |
-         (uint64_t(1) << 46) | (uint64_t(2) << 61);
+  static_assert(BK == 64 || BK == 32, "BK");
+  constexpr uint64_t kLayout = BK == 64 ? 2 : 4;
+  constexpr uint64_t kSbo = 8 * BK * 2;
+  return uint64_t((addr >> 4) & 0x3FFFu) | (uint64_t(1) << 16) | ((kSbo >> 4) << 32) |
+         (uint64_t(1) << 46) | (kLayout << 61);
 }
 // B: MN-major (W[tap] is [Cin][Cout] with Cout contiguous); 64-column blocks
 // `lbo` bytes apart, 8-row (K) groups 1024 bytes apart.
@@ -280,30 +283,40 @@ __device__ __forceinline__ int next_tap(uint32_t& rotated, int r) {
 }
 
 // One gather warp's share of a stage: which tiles it copies and from where.
-template <int G>
+template <int G, int IDX>
 struct GatherJob {
   int stage;
   uint32_t g;
   int kb;
-  uint32_t tiles;  // bit k: tile k of the group has this tap
-  int vidx[G];     // lane l: source row of local row l of tile k (-1 = zero row)
+  uint32_t tiles;    // bit k: tile k of the group has this tap
+  int vidx[G][IDX];  // lane l: source row of local row 32 i + l of tile k (-1 = zero row)
 };
 
 constexpr int kQueue = 2;  // work items published ahead of the producers (small: a
                            // reserved item cannot move to an idle SM)
 
-template <int BN, int STAGES, int G, bool BF16>
-__global__ void __launch_bounds__(threads_for(STAGES), 1)
+template <int BN, int BK, int STAGES, int G, int WPS, bool BF16>
+__global__ void __launch_bounds__(threads_for(STAGES, WPS), 1)
 k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap fmap,
           const ConvArgs args) {
   static_assert(BN % 64 == 0 && BN <= 256, "BN");
+  static_assert(BK == 64 || BK == 32, "BK");
+  constexpr int kBK = BK;
+  constexpr int kABytes = kTileRows * BK * 2;      // one tile's rows for one stage
+  constexpr int kRowBytes = BK * 2;                 // 128 or 64
+  constexpr int kChunks = kRowBytes / 16;           // 16-byte copies per row
+  constexpr int kRowsPerInstr = 32 / kChunks;       // rows one warp copy instruction covers
+  constexpr int kRowsPerWarp = kTileRows / WPS;     // rows of a tile one gather warp copies
+  constexpr int kInstr = kRowsPerWarp / kRowsPerInstr;
+  constexpr int kIdx = kRowsPerWarp / 32;           // gather indices held per lane
+  static_assert(kRowsPerWarp % 32 == 0 && kInstr >= 1, "gather split");
   constexpr int kBBytes = BN * kBK * 2;
   constexpr int kStageBytes = G * kABytes + kBBytes;
   constexpr uint32_t kTmemCols = 2 * G * BN;  // two sets of G accumulators
   constexpr uint32_t kIdesc = make_idesc(BN, BF16);
   // readers of a queue entry: gather warps, W loader, MMA thread (the epilogue
   // learns each item from the MMA thread, one accumulator at a time)
-  constexpr uint32_t kQueueReaders = kWarpsPerSlot * STAGES + 1 + 1;
+  constexpr uint32_t kQueueReaders = WPS * STAGES + 1 + 1;
   static_assert(kTmemCols >= 32 && kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0,
                 "tensor memory columns");
 
@@ -332,7 +345,7 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
     for (int s = 0; s < STAGES; ++s) {
       // sparse: the gather lanes and the W loader; dense (K = 1): the loader
       // brings the contiguous A rows with TMA too
-      mbar_init(full0 + 8 * s, args.dense ? 1 : kWarpsPerSlot * 32 + 1);
+      mbar_init(full0 + 8 * s, args.dense ? 1 : WPS * 32 + 1);
       mbar_init(empty0 + 8 * s, 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -398,17 +411,17 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
       if (w < 0) break;
     }
   } else if (warp >= kFirstGatherWarp) {
-    // ---------------- gather warps: warps 4 i .. 4 i + 3 own stage slot i ----
-    const int gw = (warp - kFirstGatherWarp) / kWarpsPerSlot;  // slot
-    const int rq = (warp - kFirstGatherWarp) % kWarpsPerSlot;  // rows 32 rq .. 32 rq + 31
-    const int chunk = lane & 7;  // 16-byte chunk within a 128-byte row slice
-    const int rsub = lane >> 3;  // instruction j copies local rows 4 j + rsub
+    // ------------- gather warps: warps WPS i .. WPS i + WPS - 1 own stage slot i ----
+    const int gw = (warp - kFirstGatherWarp) / WPS;  // slot
+    const int rq = (warp - kFirstGatherWarp) % WPS;  // rows kRowsPerWarp * rq ...
+    const int chunk = lane % kChunks;  // 16-byte chunk within a row slice
+    const int rsub = lane / kChunks;   // instruction j copies local rows kRowsPerInstr j + rsub
     // Within an item, the index loads of an owned stage are issued one owned
     // stage ahead of its copies, so they overlap the wait for the slot.
-    GatherJob<G> pend;
+    GatherJob<G, kIdx> pend;
     bool have_pend = false;
     bool ok = true;
-    auto run = [&](const GatherJob<G>& job) -> bool {
+    auto run = [&](const GatherJob<G, kIdx>& job) -> bool {
       if (!mbar_wait(empty0 + 8 * job.stage, ((job.g / STAGES) & 1) ^ 1, abort_flag,
                      args.status))
         return false;
@@ -419,12 +432,14 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
         if (!((job.tiles >> k) & 1u)) continue;
         const uint32_t a_base = stage_base + k * kABytes;
 #pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-          const int local = 4 * jj + rsub;
-          const int v = __shfl_sync(0xffffffffu, job.vidx[k], local);
-          const int row = 32 * rq + local;
+        for (int jj = 0; jj < kInstr; ++jj) {
+          const int local = kRowsPerInstr * jj + rsub;
+          const int v = __shfl_sync(0xffffffffu, job.vidx[k][local / 32], local % 32);
+          const int row = kRowsPerWarp * rq + local;
           const uint16_t* src = v >= 0 ? src_col + int64_t(v) * args.cin : args.feats;
-          cp_async_16(a_base + row * 128 + ((chunk ^ (row & 7)) << 4), src, v >= 0 ? 16u : 0u);
+          // swizzled chunk: XOR with address bits 7.. (128-byte: row & 7; 64-byte: (row >> 1) & 3)
+          const int pchunk = BK == 64 ? (chunk ^ (row & 7)) : (chunk ^ ((row >> 1) & 3));
+          cp_async_16(a_base + row * kRowBytes + (pchunk << 4), src, v >= 0 ? 16u : 0u);
         }
       }
       cp_async_arrive_noinc(full0 + 8 * job.stage);
@@ -441,18 +456,22 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
         for (int kb = 0; kb < kb_per_tap && ok; ++kb, ++g) {
           const int stage = int(g % STAGES);
           if (stage != gw) continue;
-          GatherJob<G> job;
+          GatherJob<G, kIdx> job;
           job.stage = stage;
           job.g = g;
           job.kb = kb;
           job.tiles = 0;
 #pragma unroll
           for (int k = 0; k < G; ++k) {
-            job.vidx[k] = -1;
+#pragma unroll
+            for (int i = 0; i < kIdx; ++i) job.vidx[k][i] = -1;
             if (!((cur.mask[k] >> tap) & 1u)) continue;
             job.tiles |= 1u << k;
             const int slot = cur.slot0[k] + __popc(cur.mask[k] & ((1u << tap) - 1u));
-            job.vidx[k] = args.gidx[int64_t(slot) * kTileRows + 32 * rq + lane];
+#pragma unroll
+            for (int i = 0; i < kIdx; ++i)
+              job.vidx[k][i] =
+                  args.gidx[int64_t(slot) * kTileRows + kRowsPerWarp * rq + 32 * i + lane];
           }
           if (have_pend) ok = run(pend);
           pend = job;
@@ -515,7 +534,7 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
     if (lane == 0) {
       uint32_t g = 0, j = 0, acc_iter = 0;
       bool ok = true;
-      const uint64_t adesc0 = desc_a_kmajor(smem_addr(smem));
+      const uint64_t adesc0 = desc_a_kmajor<BK>(smem_addr(smem));
       const uint64_t bdesc0 = desc_b_mnmajor(smem_addr(smem) + G * kABytes, kBK * 128);
       while (ok) {
         const Group<G> cur = next_item(j, false);
@@ -655,29 +674,32 @@ int sm_count() {
   return sms;
 }
 
-// 2-D row-major [rows][cols] tensor map with a (64 x box_rows) box and
-// 128-byte swizzle.
+// 2-D row-major [rows][cols] tensor map with a (box_cols x box_rows) box;
+// box_cols * 2 bytes is the swizzle width (128 or 64 bytes).
 bool encode_2d(CUtensorMap* map, bool bf16, const void* base, uint64_t cols, uint64_t rows,
-               uint32_t box_rows) {
+               uint32_t box_cols, uint32_t box_rows) {
   auto encode = get_encode_fn();
   if (!encode) return false;
   cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
   cuuint64_t strides[1] = {cuuint64_t(cols) * 2};
-  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle swz =
+      box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   return encode(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
                 const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, int STAGES, int G, bool BF16>
+template <int BN, int BK, int STAGES, int G, int WPS, bool BF16>
 int launch_cfg(const Plan& plan, bool dense, const void* feats, const void* W, void* out, int cin,
                int cout, cudaStream_t stream) {
-  constexpr int kStageBytes = G * kABytes + BN * kBK * 2;
+  constexpr int kStageBytes = G * kTileRows * BK * 2 + BN * BK * 2;
   constexpr int kSmem = STAGES * kStageBytes + 1024 + 512;
   static_assert(kSmem <= 227 * 1024, "shared memory");
-  auto kern = k_conv_tc<BN, STAGES, G, BF16>;
+  static_assert(threads_for(STAGES, WPS) <= 1024, "threads");
+  auto kern = k_conv_tc<BN, BK, STAGES, G, WPS, BF16>;
   static bool attr_set = false;
   if (!attr_set) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) !=
@@ -687,8 +709,8 @@ int launch_cfg(const Plan& plan, bool dense, const void* feats, const void* W, v
   }
   CUtensorMap wmap, fmap;
   const int taps = dense ? 1 : kTaps;
-  if (!encode_2d(&wmap, BF16, W, uint64_t(cout), uint64_t(taps) * uint64_t(cin), kBK) ||
-      !encode_2d(&fmap, BF16, feats, uint64_t(cin), uint64_t(plan.n), kTileRows))
+  if (!encode_2d(&wmap, BF16, W, uint64_t(cout), uint64_t(taps) * uint64_t(cin), 64, BK) ||
+      !encode_2d(&fmap, BF16, feats, uint64_t(cin), uint64_t(plan.n), BK, kTileRows))
     return SMC_ERR_CUDA;
   ConvArgs a;
   a.feats = static_cast<const uint16_t*>(feats);
@@ -710,39 +732,52 @@ int launch_cfg(const Plan& plan, bool dense, const void* feats, const void* W, v
     return SMC_ERR_CUDA;
   const int64_t work = int64_t(a.n_groups) * a.n_blocks;
   const int grid = int(std::min<int64_t>(work, sm_count()));
-  kern<<<grid, threads_for(STAGES), kSmem, stream>>>(wmap, fmap, a);
+  kern<<<grid, threads_for(STAGES, WPS), kSmem, stream>>>(wmap, fmap, a);
   return cudaGetLastError() == cudaSuccess ? SMC_OK : SMC_ERR_CUDA;
 }
 
-// Tile-group size override for tuning (SMC_TC_GROUP=1 or 2; default 2 for
-// BN < 256), read once.
+// Tuning overrides, read once per process: SMC_TC_GROUP=1 (one tile per work
+// item) and SMC_TC_BK=32 (32-channel stages, twice as many, 64-byte swizzle).
+int env_int(const char* name) {
+  const char* e = std::getenv(name);
+  return e ? std::atoi(e) : 0;
+}
 int group_override() {
-  static int v = [] {
-    const char* e = std::getenv("SMC_TC_GROUP");
-    return e ? std::atoi(e) : 0;
-  }();
+  static int v = env_int("SMC_TC_GROUP");
+  return v;
+}
+int bk_override() {
+  static int v = env_int("SMC_TC_BK");
   return v;
 }
 
 template <bool BF16>
 int launch_dtype(const Plan& plan, bool dense, const void* feats, const void* W, void* out,
                  int cin, int cout, cudaStream_t stream) {
+  //            BN  BK  stages G WPS
+  if (bk_override() == 32) {
+    if (cout % 256 == 0)
+      return launch_cfg<256, 32, 8, 1, 2, BF16>(plan, dense, feats, W, out, cin, cout, stream);
+    if (cout % 128 == 0)
+      return launch_cfg<128, 32, 8, 2, 2, BF16>(plan, dense, feats, W, out, cin, cout, stream);
+    return launch_cfg<64, 32, 10, 2, 2, BF16>(plan, dense, feats, W, out, cin, cout, stream);
+  }
   if (group_override() == 1 && cout % 256 != 0) {
     if (cout % 128 == 0)
-      return launch_cfg<128, 5, 1, BF16>(plan, dense, feats, W, out, cin, cout, stream);
-    return launch_cfg<64, 6, 1, BF16>(plan, dense, feats, W, out, cin, cout, stream);
+      return launch_cfg<128, 64, 5, 1, 4, BF16>(plan, dense, feats, W, out, cin, cout, stream);
+    return launch_cfg<64, 64, 6, 1, 4, BF16>(plan, dense, feats, W, out, cin, cout, stream);
   }
   if (cout % 256 == 0)
-    return launch_cfg<256, 4, 1, BF16>(plan, dense, feats, W, out, cin, cout, stream);
+    return launch_cfg<256, 64, 4, 1, 4, BF16>(plan, dense, feats, W, out, cin, cout, stream);
   if (cout % 128 == 0)
-    return launch_cfg<128, 4, 2, BF16>(plan, dense, feats, W, out, cin, cout, stream);
-  return launch_cfg<64, 5, 2, BF16>(plan, dense, feats, W, out, cin, cout, stream);
+    return launch_cfg<128, 64, 4, 2, 4, BF16>(plan, dense, feats, W, out, cin, cout, stream);
+  return launch_cfg<64, 64, 5, 2, 4, BF16>(plan, dense, feats, W, out, cin, cout, stream);
 }
 
 }  // namespace
 
 bool conv_tc_supported(int cin, int cout, int dtype) {
-  return (dtype == SMC_F16 || dtype == SMC_BF16) && cin > 0 && cout > 0 && cin % kBK == 0 &&
+  return (dtype == SMC_F16 || dtype == SMC_BF16) && cin > 0 && cout > 0 && cin % 64 == 0 &&
          cout % 64 == 0;
 }
 

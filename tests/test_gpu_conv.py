@@ -178,29 +178,36 @@ sys.path.insert(0, {root!r}); sys.path.insert(0, {tests!r})
 from submanifold_sparse_convolution_coord_b200 import synth
 from submanifold_sparse_convolution_coord_b200.binding import SubMIndex
 from gpu_common import check_conv, oracle_conv
-cases = [(0, 3000, 20, 1, 128, 128, "f16"), (1, 800, 40, 2, 64, 64, "bf16"), (2, 2000, 16, 1, 64, 128, "f16")]
+cases = [(0, 3000, 20, 1, 128, 128, "f16"), (1, 800, 40, 2, 64, 64, "bf16"), (2, 2000, 16, 1, 64, 128, "f16"),
+         (3, 900, 14, 1, 192, 256, "bf16"), (4, 1500, 30, 2, 128, 64, "f16")]
 for seed, n, grid, batch, cin, cout, dt in cases:
     coords, feats, W = synth.random_case(seed, n, grid, batch, cin, cout, 3, dt, True)
     idx = SubMIndex(torch.from_numpy(coords).cuda())
     out = idx.forward(feats.cuda(), W.cuda())
+    W1 = synth.round_to(np.random.default_rng(seed).standard_normal((1, cin, cout)) / cin ** 0.5, dt)
+    out1 = idx.forward(feats.cuda(), W1.cuda(), K=1)
     torch.cuda.synchronize()
     assert idx.status() == 0
     ref, scale = oracle_conv(coords, feats, W, 3)
     check_conv(out, ref, scale, str((seed, cin, cout)))
+    ref1, scale1 = oracle_conv(coords, feats, W1, 1)
+    check_conv(out1, ref1, scale1, str((seed, cin, cout, "K1")))
     idx.close()
 print("ok")
 """
 
 
-def test_group_size_one_configuration():
-    """The tile-group-size override (one tile per work item) in a fresh
-    process, since the setting is read once per process."""
+@pytest.mark.parametrize("override", [("SMC_TC_GROUP", "1"), ("SMC_TC_BK", "32")])
+def test_tuning_override_configurations(override):
+    """The kernel configurations behind the tuning overrides (one tile per work
+    item; 32-channel stages with 64-byte swizzle), each in a fresh process
+    since the settings are read once per process."""
     import os
     import subprocess
     import sys
     here = os.path.dirname(os.path.abspath(__file__))
     code = _GROUP1_SCRIPT.format(root=os.path.dirname(here), tests=here)
-    env = dict(os.environ, SMC_TC_GROUP="1")
+    env = dict(os.environ, **{override[0]: override[1]})
     r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True,
                        timeout=600)
     assert r.returncode == 0 and "ok" in r.stdout, r.stdout + r.stderr
