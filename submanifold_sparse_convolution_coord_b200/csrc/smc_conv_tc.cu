@@ -223,7 +223,7 @@ struct ConvArgs {
   const int32_t* tile_off;    // [n_tiles + 1] first slot of each tile
   const uint32_t* tile_mask;  // [n_tiles] active taps of each tile
   const int32_t* out_row;     // [n_tiles * 128], -1 = padding row
-  uint32_t* work_counter;     // zeroed before the launch
+  uint32_t* work_counter;     // [0] next item, [1] CTAs finished; both 0 between launches
   int32_t* status;
   int64_t n;
   int cin;
@@ -646,6 +646,15 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
+  // The last CTA to finish resets the item counter for the next launch (every
+  // CTA's last atomicAdd on it happened before it got here).
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(args.work_counter + 1, 1u) == gridDim.x - 1) {
+      atomicExch(args.work_counter, 0u);
+      atomicExch(args.work_counter + 1, 0u);
+    }
+  }
 }
 
 // ----------------------------------------------------------------------------
@@ -666,11 +675,19 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   return fn;
 }
 
+// SM count of the current device, cached per device.
 int sm_count() {
-  int dev = 0, sms = 0;
+  constexpr int kMaxDev = 64;
+  static int cache[kMaxDev] = {};
+  int dev = 0;
   cudaGetDevice(&dev);
-  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+  if (dev >= 0 && dev < kMaxDev && cache[dev] > 0) return cache[dev];
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) {
+    cudaGetLastError();
     sms = 148;
+  }
+  if (dev >= 0 && dev < kMaxDev) cache[dev] = sms;
   return sms;
 }
 
@@ -727,17 +744,16 @@ int launch_cfg(const Plan& plan, bool dense, const void* feats, const void* W, v
   a.n_blocks = cout / BN;
   a.n_groups = int((plan.n_tiles + G - 1) / G);
   a.dense = dense ? 1 : 0;
-  a.work_counter = plan.work_counter;
-  if (cudaMemsetAsync(plan.work_counter, 0, sizeof(uint32_t), stream) != cudaSuccess)
-    return SMC_ERR_CUDA;
+  a.work_counter = plan.work_counter;  // zero since the build; reset by each launch
   const int64_t work = int64_t(a.n_groups) * a.n_blocks;
   const int grid = int(std::min<int64_t>(work, sm_count()));
   kern<<<grid, threads_for(STAGES, WPS), kSmem, stream>>>(wmap, fmap, a);
   return cudaGetLastError() == cudaSuccess ? SMC_OK : SMC_ERR_CUDA;
 }
 
-// Tuning overrides, read once per process: SMC_TC_GROUP=1 (one tile per work
-// item) and SMC_TC_BK=32 (32-channel stages, twice as many, 64-byte swizzle).
+// Tuning overrides, read once per process: SMC_TC_GROUP=1 or 2 (tiles per work
+// item, default: 1 below 6 tiles per SM, else 2) and SMC_TC_BK=32 (32-channel
+// stages, twice as many, 64-byte swizzle).
 int env_int(const char* name) {
   const char* e = std::getenv(name);
   return e ? std::atoi(e) : 0;
@@ -754,6 +770,9 @@ int bk_override() {
 template <bool BF16>
 int launch_dtype(const Plan& plan, bool dense, const void* feats, const void* W, void* out,
                  int cin, int cout, cudaStream_t stream) {
+  // Few tiles per SM: one tile per work item, so every SM gets work and no SM
+  // runs two heavy tiles back to back.
+  const bool small = plan.n_tiles < int64_t(6) * sm_count();
   //            BN  BK  stages G WPS
   if (bk_override() == 32) {
     if (cout % 256 == 0)
@@ -762,7 +781,7 @@ int launch_dtype(const Plan& plan, bool dense, const void* feats, const void* W,
       return launch_cfg<128, 32, 8, 2, 2, BF16>(plan, dense, feats, W, out, cin, cout, stream);
     return launch_cfg<64, 32, 10, 2, 2, BF16>(plan, dense, feats, W, out, cin, cout, stream);
   }
-  if (group_override() == 1 && cout % 256 != 0) {
+  if ((group_override() == 1 || (small && group_override() != 2)) && cout % 256 != 0) {
     if (cout % 128 == 0)
       return launch_cfg<128, 64, 5, 1, 4, BF16>(plan, dense, feats, W, out, cin, cout, stream);
     return launch_cfg<64, 64, 6, 1, 4, BF16>(plan, dense, feats, W, out, cin, cout, stream);

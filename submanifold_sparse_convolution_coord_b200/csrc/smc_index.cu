@@ -340,6 +340,8 @@ int build_plan_impl(const int32_t* coords, int64_t n, int32_t stride, int64_t ta
   const int4* c4 = reinterpret_cast<const int4*>(coords);
   SMC_TRY(dev_alloc(&plan->status, 1, s));
   SMC_TRY(dev_alloc(&plan->work_counter, 64, s));
+  if (cudaMemsetAsync(plan->work_counter, 0, 64 * sizeof(uint32_t), s) != cudaSuccess)
+    return SMC_ERR_CUDA;
   if (cudaMemsetAsync(plan->status, 0, sizeof(int32_t), s) != cudaSuccess) return SMC_ERR_CUDA;
   plan->n = n;
   plan->n_tiles = (n + kTileRows - 1) / kTileRows;

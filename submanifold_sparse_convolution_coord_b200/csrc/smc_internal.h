@@ -36,7 +36,7 @@ struct Plan {
   int32_t* gidx = nullptr;        // [total_slots][128] voxel gathered per row, -1 = none
   int32_t* out_row = nullptr;     // [n_tiles * 128] voxel written per plan row, -1 = none
   int32_t* status = nullptr;      // device status word
-  uint32_t* work_counter = nullptr;  // tensor-core kernel's item counter, zeroed per launch
+  uint32_t* work_counter = nullptr;  // tensor-core kernel's item counter (+ finished CTAs)
   int64_t useful_pairs = 0;
   int64_t issued_rows_taps = 0;
 };
