@@ -197,7 +197,8 @@ print("ok")
 """
 
 
-@pytest.mark.parametrize("override", [("SMC_TC_GROUP", "1"), ("SMC_TC_BK", "32")])
+@pytest.mark.parametrize("override", [("SMC_TC_GROUP", "1"), ("SMC_TC_GROUP", "2"),
+                                      ("SMC_TC_BK", "32")])
 def test_tuning_override_configurations(override):
     """The kernel configurations behind the tuning overrides (one tile per work
     item; 32-channel stages with 64-byte swizzle), each in a fresh process
