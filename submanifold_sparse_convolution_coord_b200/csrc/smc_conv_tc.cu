@@ -295,7 +295,9 @@ struct GatherJob {
 constexpr int kQueue = 2;  // work items published ahead of the producers (small: a
                            // reserved item cannot move to an idle SM)
 
-template <int BN, int BK, int STAGES, int G, int WPS, bool BF16>
+// NBUF: accumulator sets in tensor memory (2: the epilogue of one item overlaps
+// the MMAs of the next; 1: room for two 256-column tiles per item).
+template <int BN, int BK, int STAGES, int G, int WPS, bool BF16, int NBUF>
 __global__ void __launch_bounds__(threads_for(STAGES, WPS), 1)
 k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap fmap,
           const ConvArgs args) {
@@ -312,7 +314,8 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
   static_assert(kRowsPerWarp % 32 == 0 && kInstr >= 1, "gather split");
   constexpr int kBBytes = BN * kBK * 2;
   constexpr int kStageBytes = G * kABytes + kBBytes;
-  constexpr uint32_t kTmemCols = 2 * G * BN;  // two sets of G accumulators
+  static_assert(NBUF == 1 || NBUF == 2, "accumulator sets");
+  constexpr uint32_t kTmemCols = NBUF * G * BN;  // NBUF sets of G accumulators
   constexpr uint32_t kIdesc = make_idesc(BN, BF16);
   // readers of a queue entry: gather warps, W loader, MMA thread (the epilogue
   // learns each item from the MMA thread, one accumulator at a time)
@@ -538,8 +541,9 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
       const uint64_t bdesc0 = desc_b_mnmajor(smem_addr(smem) + G * kABytes, kBK * 128);
       while (ok) {
         const Group<G> cur = next_item(j, false);
-        const uint32_t a = acc_iter & 1;
-        if (!mbar_wait(tempty0 + 8 * a, ((acc_iter >> 1) & 1) ^ 1, abort_flag, args.status)) {
+        const uint32_t a = acc_iter % NBUF;
+        const uint32_t use = acc_iter / NBUF;  // how many times set a was used before
+        if (!mbar_wait(tempty0 + 8 * a, (use & 1) ^ 1, abort_flag, args.status)) {
           ok = false;
           break;
         }
@@ -579,7 +583,7 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
           }
         }
         umma_commit(tfull0 + 8 * a);
-        if (!ok) mbar_drain(tfull0 + 8 * a, (acc_iter >> 1) & 1);
+        if (!ok) mbar_drain(tfull0 + 8 * a, use & 1);
         ++acc_iter;
       }
     }
@@ -590,8 +594,9 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
     const int row = quarter * 32 + lane;
     uint32_t acc_iter = 0;
     while (true) {
-      const uint32_t a = acc_iter & 1;
-      bool have = mbar_wait(info0 + 8 * a, (acc_iter >> 1) & 1, abort_flag, args.status);
+      const uint32_t a = acc_iter % NBUF;
+      const uint32_t use = acc_iter / NBUF;
+      bool have = mbar_wait(info0 + 8 * a, use & 1, abort_flag, args.status);
       have = __all_sync(0xffffffffu, have);
       if (!have) break;
       const Group<G> gr = acc_info[a];
@@ -607,7 +612,7 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
         else
           orow[k] = args.out_row[r];
       }
-      have = mbar_wait(tfull0 + 8 * a, (acc_iter >> 1) & 1, abort_flag, args.status);
+      have = mbar_wait(tfull0 + 8 * a, use & 1, abort_flag, args.status);
       have = __all_sync(0xffffffffu, have);  // tcgen05.ld below is warp-collective
       if (!have) break;
       tc_fence_after();
@@ -709,14 +714,14 @@ bool encode_2d(CUtensorMap* map, bool bf16, const void* base, uint64_t cols, uin
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, int BK, int STAGES, int G, int WPS, bool BF16>
+template <int BN, int BK, int STAGES, int G, int WPS, bool BF16, int NBUF = 2>
 int launch_cfg(const Plan& plan, bool dense, const void* feats, const void* W, void* out, int cin,
                int cout, cudaStream_t stream) {
   constexpr int kStageBytes = G * kTileRows * BK * 2 + BN * BK * 2;
   constexpr int kSmem = STAGES * kStageBytes + 1024 + 512;
   static_assert(kSmem <= 227 * 1024, "shared memory");
   static_assert(threads_for(STAGES, WPS) <= 1024, "threads");
-  auto kern = k_conv_tc<BN, BK, STAGES, G, WPS, BF16>;
+  auto kern = k_conv_tc<BN, BK, STAGES, G, WPS, BF16, NBUF>;
   static bool attr_set = false;
   if (!attr_set) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) !=
@@ -786,8 +791,16 @@ int launch_dtype(const Plan& plan, bool dense, const void* feats, const void* W,
       return launch_cfg<128, 64, 5, 1, 4, BF16>(plan, dense, feats, W, out, cin, cout, stream);
     return launch_cfg<64, 64, 6, 1, 4, BF16>(plan, dense, feats, W, out, cin, cout, stream);
   }
-  if (cout % 256 == 0)
+  if (cout % 256 == 0) {
+    // sparse: two 256-column tiles per item share each W slice (single
+    // accumulator set), as long as that leaves at least two items per SM;
+    // dense (K = 1) items are short, so they keep the overlapped epilogue
+    const int64_t items2 = (plan.n_tiles + 1) / 2 * (cout / 256);
+    if (group_override() == 2 ||
+        (group_override() == 0 && !dense && items2 >= 2 * int64_t(sm_count())))
+      return launch_cfg<256, 64, 3, 2, 4, BF16, 1>(plan, dense, feats, W, out, cin, cout, stream);
     return launch_cfg<256, 64, 4, 1, 4, BF16>(plan, dense, feats, W, out, cin, cout, stream);
+  }
   if (cout % 128 == 0)
     return launch_cfg<128, 64, 4, 2, 4, BF16>(plan, dense, feats, W, out, cin, cout, stream);
   return launch_cfg<64, 64, 5, 2, 4, BF16>(plan, dense, feats, W, out, cin, cout, stream);
