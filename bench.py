@@ -45,7 +45,10 @@ DTYPE_NAME = {"f16": "f16", "bf16": "bf16", "f32": "f32"}
 # dram__bytes_read.sum + dram__bytes_write.sum of one k_conv_tc launch, from the
 # ncu capture summarised in profiles/k_conv_tc_<workload>.md (bytes).  Only
 # workloads captured with the current kernel are listed; others report null.
-NCU_TRAFFIC = {"uniform128": 66.160128e6 + 14.779904e6}
+NCU_TRAFFIC = {"uniform128": 65.874688e6 + 14.860032e6}
+# fp32 features run on the CUDA cores with fp64 accumulation: the ALU bound is
+# the fp64 FMA rate, 148 SMs x 64 fp64 lanes x 2 FLOP x 1.965 GHz.
+FP64_ALU_TFLOPS = 148 * 64 * 2 * 1.965e9 / 1e12
 
 
 def load_peaks() -> tuple:
@@ -334,8 +337,10 @@ def run_ours(args) -> None:
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": conv_ms_max,
         "higher_is_better": True, "scaling": "weak",
-        # the README's 13.8 ms for this layer, as useful TFLOP/s on the same pairs
-        "vs_baseline": value / (flops_all / (PAGES_CONV_MS * 1e-3) / 1e12),
+        # the README's 13.8 ms for this layer (M3 Ultra), as useful TFLOP/s on
+        # the same pairs; the pages time no other workload
+        "vs_baseline": (value / (flops_all / (PAGES_CONV_MS * 1e-3) / 1e12)
+                        if args.workload == "uniform128" else None),
         "dtype": DTYPE_NAME[w.dtype], "data": "synthetic",
         "config": {"workload": args.workload, "grid": w.grid, "batch": w.batch,
                    "n_voxels": inp.n, "cin": cin, "cout": cout, "K": 3,
@@ -345,11 +350,15 @@ def run_ours(args) -> None:
         "conv_ms": conv_ms_max,
         "conv_ms_p50": float(np.median(per)),
         "index_build_ms": float(np.median(build_ms)),
-        "useful_pairs": pairs, "issued_rows_taps": issued,
-        "useful_fraction": pairs / issued if issued else None,
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": NCU_TRAFFIC.get(args.workload),
-                     "peak_source": f"bf16 dense burst, {peak_kind} (fp16 assumed equal)",
+        "useful_pairs": pairs, "issued_rows_taps": issued if w.dtype != "f32" else None,
+        "useful_fraction": (pairs / issued if issued else None) if w.dtype != "f32" else None,
+        "roofline": {"bound": "tensor" if w.dtype != "f32" else "alu", "achieved": achieved,
+                     "peak": peak if w.dtype != "f32" else FP64_ALU_TFLOPS, "unit": "TFLOP/s",
+                     "frac": achieved / (peak if w.dtype != "f32" else FP64_ALU_TFLOPS),
+                     "traffic": NCU_TRAFFIC.get(args.workload),
+                     "peak_source": (f"bf16 dense burst, {peak_kind} (fp16 assumed equal)"
+                                     if w.dtype != "f32" else
+                                     "fp64 FMA: 148 SMs x 64 lanes x 2 x 1.965 GHz"),
                      "algorithmic_bytes": algo_bytes,
                      "hbm_gbs_algorithmic": algo_bytes / (conv_ms * 1e-3) / 1e9,
                      "hbm_frac": algo_bytes / (conv_ms * 1e-3) / 1e9 / hbm_peak},
