@@ -10,19 +10,24 @@
 // organised so that the dense work of the README's fused
 // [N, 27 Cin] x [27 Cin, Cout] matmul is skipped one tile-tap at a time.
 //
-// Persistent kernel, one CTA per SM, 7 + 4 * STAGES warps:
+// Persistent kernel, one CTA per SM, 8 + WPS * STAGES warps:
 //   warp 0      lane 0 loads the W[tap] slice of each stage with TMA
 //               (MN-major, 128-byte swizzle), and for K = 1 also the stage's
 //               contiguous feature rows (128 x 64 box, 128-byte swizzle);
-//   warp 1      allocates tensor memory; lane 0 issues the MMAs (M = 128,
-//               N = BN, K = 16) into one of two accumulators;
+//   warp 1      allocates tensor memory; with the last warp, issues the MMAs
+//               (M = 128, N = BN, K = 16): warp 1 those of the even tiles of
+//               a work item, the last warp those of the odd tiles.  A
+//               tcgen05.mma keeps its issuing thread until the tensor core
+//               accepts it (about one MMA time), so a single issuer's own
+//               loop and waits between stages would idle the tensor core;
+//               two issuers cover each other's gaps;
 //   warps 2-5   epilogue: tensor memory -> registers -> fp16/bf16 -> global,
 //               overlapping the MMAs of the next work item;
 //   warp 6      scheduler: takes work items (heaviest first) from a global
 //               counter and decodes each one's tile masks and slot offsets
 //               into a small shared-memory queue read by every other role;
-//   warps 7..   gather, four warps per pipeline stage slot: warp q of slot i
-//               copies rows 32 q .. 32 q + 31 of every tile the stage feeds
+//   warps 7..   gather, WPS (4 or 2) warps per pipeline stage slot: warp q of
+//               slot i copies rows 128/WPS q .. of every tile the stage feeds
 //               (64 channels, 128 bytes per row) with 16-byte cp.async
 //               (zero-filled for absent neighbours) into a 128-byte-swizzled
 //               K-major tile; each lane's mbarrier arrival fires when its
@@ -49,9 +54,11 @@ namespace {
 
 constexpr int kPrefetchWarp = 6;
 constexpr int kFirstGatherWarp = 7;
-// gather warps per stage slot (each copies 128 / WPS of a tile's rows)
+// Warps: 0 W loader, 1 MMA (even tiles of a group), 2-5 epilogue, 6 scheduler,
+// then WPS gather warps per stage slot (each copies 128 / WPS of a tile's
+// rows), then the second MMA warp (odd tiles).
 __host__ __device__ constexpr int threads_for(int stages, int wps) {
-  return 32 * (kFirstGatherWarp + wps * stages);
+  return 32 * (kFirstGatherWarp + wps * stages + 1);
 }
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
@@ -317,9 +324,16 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
   static_assert(NBUF == 1 || NBUF == 2, "accumulator sets");
   constexpr uint32_t kTmemCols = NBUF * G * BN;  // NBUF sets of G accumulators
   constexpr uint32_t kIdesc = make_idesc(BN, BF16);
-  // readers of a queue entry: gather warps, W loader, MMA thread (the epilogue
-  // learns each item from the MMA thread, one accumulator at a time)
-  constexpr uint32_t kQueueReaders = WPS * STAGES + 1 + 1;
+  // Two MMA warps: a tcgen05.mma holds its issuing thread until the tensor core
+  // takes it, so one issuer's own loop and barrier waits would leave the tensor
+  // core idle between stages.  Warp 1 issues the even tiles of a group, the
+  // last warp the odd ones (separate accumulators, so no ordering between
+  // them is needed); both commit every stage.
+  constexpr int kMmaWarp2 = kFirstGatherWarp + WPS * STAGES;
+  constexpr uint32_t kMmaWarps = 2;
+  // readers of a queue entry: gather warps, W loader, both MMA warps (the
+  // epilogue learns each item from MMA warp 1, one accumulator at a time)
+  constexpr uint32_t kQueueReaders = WPS * STAGES + 1 + kMmaWarps;
   static_assert(kTmemCols >= 32 && kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0,
                 "tensor memory columns");
 
@@ -349,10 +363,10 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
       // sparse: the gather lanes and the W loader; dense (K = 1): the loader
       // brings the contiguous A rows with TMA too
       mbar_init(full0 + 8 * s, args.dense ? 1 : WPS * 32 + 1);
-      mbar_init(empty0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, kMmaWarps);
     }
     for (int a = 0; a < 2; ++a) {
-      mbar_init(tfull0 + 8 * a, 1);
+      mbar_init(tfull0 + 8 * a, kMmaWarps);
       mbar_init(tempty0 + 8 * a, 4 * 32);
       mbar_init(info0 + 8 * a, 1);
     }
@@ -413,7 +427,7 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
       }
       if (w < 0) break;
     }
-  } else if (warp >= kFirstGatherWarp) {
+  } else if (warp >= kFirstGatherWarp && warp < kMmaWarp2) {
     // ------------- gather warps: warps WPS i .. WPS i + WPS - 1 own stage slot i ----
     const int gw = (warp - kFirstGatherWarp) / WPS;  // slot
     const int rq = (warp - kFirstGatherWarp) % WPS;  // rows kRowsPerWarp * rq ...
@@ -425,6 +439,15 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
     bool have_pend = false;
     bool ok = true;
     auto run = [&](const GatherJob<G, kIdx>& job) -> bool {
+      // the source row of every copy, exchanged before the wait for the slot
+      int vv[G][kInstr];
+#pragma unroll
+      for (int k = 0; k < G; ++k)
+#pragma unroll
+        for (int jj = 0; jj < kInstr; ++jj) {
+          const int local = kRowsPerInstr * jj + rsub;
+          vv[k][jj] = __shfl_sync(0xffffffffu, job.vidx[k][local / 32], local % 32);
+        }
       if (!mbar_wait(empty0 + 8 * job.stage, ((job.g / STAGES) & 1) ^ 1, abort_flag,
                      args.status))
         return false;
@@ -437,7 +460,7 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
 #pragma unroll
         for (int jj = 0; jj < kInstr; ++jj) {
           const int local = kRowsPerInstr * jj + rsub;
-          const int v = __shfl_sync(0xffffffffu, job.vidx[k][local / 32], local % 32);
+          const int v = vv[k][jj];
           const int row = kRowsPerWarp * rq + local;
           const uint16_t* src = v >= 0 ? src_col + int64_t(v) * args.cin : args.feats;
           // swizzled chunk: XOR with address bits 7.. (128-byte: row & 7; 64-byte: (row >> 1) & 3)
@@ -483,7 +506,7 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
       }
       // Never carry a stage into the next item: the next owned stage may lie
       // several items ahead, which the queue only publishes once the MMA
-      // thread has moved on -- and the MMA thread waits for this stage.
+      // warps have moved on -- and the MMA warps wait for this stage.
       if (have_pend && ok) ok = run(pend);
       have_pend = false;
     }
@@ -532,44 +555,51 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
-      uint32_t g = 0, j = 0, acc_iter = 0;
-      bool ok = true;
-      const uint64_t adesc0 = desc_a_kmajor<BK>(smem_addr(smem));
-      const uint64_t bdesc0 = desc_b_mnmajor(smem_addr(smem) + G * kABytes, kBK * 128);
-      while (ok) {
-        const Group<G> cur = next_item(j, false);
-        const uint32_t a = acc_iter % NBUF;
-        const uint32_t use = acc_iter / NBUF;  // how many times set a was used before
-        if (!mbar_wait(tempty0 + 8 * a, (use & 1) ^ 1, abort_flag, args.status)) {
-          ok = false;
-          break;
-        }
-        // tell the epilogue which item this accumulator will hold (or that
-        // there are no more); the buffer's epilogue has finished with it
+  } else if (warp == 1 || warp == kMmaWarp2) {
+    // ---------------- MMA warps ----------------
+    // The whole warp runs the loop (waits, item bookkeeping); lane 0 issues.
+    const int mine = warp == 1 ? 0 : 1;  // this warp's tiles: k % 2 == mine
+    uint32_t g = 0, j = 0, acc_iter = 0;
+    bool ok = true;
+    const uint64_t adesc0 = desc_a_kmajor<BK>(smem_addr(smem));
+    const uint64_t bdesc0 = desc_b_mnmajor(smem_addr(smem) + G * kABytes, kBK * 128);
+    while (ok) {
+      const Group<G> cur = next_item(j, true);
+      const uint32_t a = acc_iter % NBUF;
+      const uint32_t use = acc_iter / NBUF;  // how many times set a was used before
+      const bool free = mbar_wait(tempty0 + 8 * a, (use & 1) ^ 1, abort_flag, args.status);
+      if (!__all_sync(0xffffffffu, free)) break;
+      // tell the epilogue which item this accumulator will hold (or that there
+      // are no more); the buffer's epilogue has finished with it
+      if (mine == 0 && lane == 0) {
         acc_info[a] = cur;
         mbar_arrive(info0 + 8 * a);
-        if (cur.w < 0) break;
-        tc_fence_after();
-        uint32_t started = 0;  // bit k: tile k's accumulator holds a partial sum
-        uint32_t rem = rotate_taps(cur.all, cur.rot);
-        while (rem && ok) {
-          const int tap = next_tap(rem, cur.rot);
-          for (int kb = 0; kb < kb_per_tap; ++kb, ++g) {
-            const int stage = int(g % STAGES);
-            if (!mbar_wait(full0 + 8 * stage, (g / STAGES) & 1, abort_flag, args.status)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
+      }
+      __syncwarp();
+      if (cur.w < 0) break;
+      tc_fence_after();
+      uint32_t started = 0;  // bit k: tile k's accumulator holds a partial sum
+      uint32_t rem = rotate_taps(cur.all, cur.rot);
+      while (rem && ok) {
+        const int tap = next_tap(rem, cur.rot);
+        uint32_t live = 0;  // tiles of the group that have this tap
+#pragma unroll
+        for (int k = 0; k < G; ++k) live |= ((cur.mask[k] >> tap) & 1u) << k;
+        for (int kb = 0; kb < kb_per_tap; ++kb, ++g) {
+          const int stage = int(g % STAGES);
+          const bool ready = mbar_wait(full0 + 8 * stage, (g / STAGES) & 1, abort_flag, args.status);
+          if (!__all_sync(0xffffffffu, ready)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (lane == 0) {
             // descriptors of this stage: the start-address field (bits 0-13,
             // 16-byte units) never carries, so offsets add to the 64-bit value
             const uint64_t soff = uint64_t(stage) * (kStageBytes >> 4);
 #pragma unroll
             for (int k = 0; k < G; ++k) {
-              if (!((cur.mask[k] >> tap) & 1u)) continue;
+              if (!((live >> k) & 1u) || (k & 1) != mine) continue;
               const uint32_t d_tmem = tmem + (a * G + k) * BN;
               const uint64_t ad = adesc0 + soff + uint64_t(k * (kABytes >> 4));
               const uint64_t bd = bdesc0 + soff;
@@ -577,17 +607,18 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
 #pragma unroll
               for (int kk = 0; kk < kBK / 16; ++kk)
                 umma_f16(d_tmem, ad + 2 * kk, bd + (2048 >> 4) * kk, kIdesc, kk != 0 ? 1u : acc);
-              started |= 1u << k;
             }
             umma_commit(empty0 + 8 * stage);
           }
+          __syncwarp();
+          started |= live;
         }
-        umma_commit(tfull0 + 8 * a);
-        if (!ok) mbar_drain(tfull0 + 8 * a, use & 1);
-        ++acc_iter;
       }
+      if (lane == 0) umma_commit(tfull0 + 8 * a);
+      __syncwarp();
+      if (!ok) mbar_drain(tfull0 + 8 * a, use & 1);
+      ++acc_iter;
     }
-    __syncwarp();
   } else {
     // ---------------- epilogue (warps 2-5) ----------------
     const int quarter = warp & 3;  // tensor-memory lanes 32*quarter .. +31
