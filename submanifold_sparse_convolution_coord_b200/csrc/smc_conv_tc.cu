@@ -299,9 +299,6 @@ struct GatherJob {
   int vidx[G][IDX];  // lane l: source row of local row 32 i + l of tile k (-1 = zero row)
 };
 
-constexpr int kQueue = 2;  // work items published ahead of the producers (small: a
-                           // reserved item cannot move to an idle SM)
-
 // NBUF: accumulator sets in tensor memory (2: the epilogue of one item overlaps
 // the MMAs of the next; 1: room for two 256-column tiles per item).
 template <int BN, int BK, int STAGES, int G, int WPS, bool BF16, int NBUF>
@@ -330,6 +327,12 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
   // last warp the odd ones (separate accumulators, so no ordering between
   // them is needed); both commit every stage.
   constexpr int kMmaWarp2 = kFirstGatherWarp + WPS * STAGES;
+  // Work items published ahead of the producers.  An item taken from the
+  // global counter cannot move to an idle SM any more, so a deeper queue
+  // leaves a longer tail: one entry for the 64/128-column tiles (many short
+  // items); two for 256-column tiles, whose long items would otherwise wait
+  // for the scheduler's decode at every item boundary.
+  constexpr int kQueue = BN == 256 ? 2 : 1;
   constexpr uint32_t kMmaWarps = 2;
   // readers of a queue entry: gather warps, W loader, both MMA warps (the
   // epilogue learns each item from MMA warp 1, one accumulator at a time)
