@@ -158,19 +158,28 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
                : "memory");
 }
+// MMA issue and commit, called by all 32 lanes of a converged warp: elect.sync
+// picks one lane (the same one every time, lane 0, as all lanes are active),
+// which issues.  Keeping the warp converged lets the operands stay warp-uniform;
+// the same lane issues every MMA and commit, as a commit tracks the MMAs of its
+// own thread.
 __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                          uint32_t idesc, uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   bar)
-               : "memory");
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+          bar)
+      : "memory");
 }
 __device__ __forceinline__ void tmem_ld_x32(uint32_t taddr, uint32_t (&v)[32]) {
   asm volatile(
@@ -560,7 +569,8 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
     __syncwarp();
   } else if (warp == 1 || warp == kMmaWarp2) {
     // ---------------- MMA warps ----------------
-    // The whole warp runs the loop (waits, item bookkeeping); lane 0 issues.
+    // The whole warp runs the loop (waits, item bookkeeping, descriptors) and
+    // stays converged; one elected lane issues.
     const int mine = warp == 1 ? 0 : 1;  // this warp's tiles: k % 2 == mine
     uint32_t g = 0, j = 0, acc_iter = 0;
     bool ok = true;
@@ -596,7 +606,7 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
             break;
           }
           tc_fence_after();
-          if (lane == 0) {
+          {
             // descriptors of this stage: the start-address field (bits 0-13,
             // 16-byte units) never carries, so offsets add to the 64-bit value
             const uint64_t soff = uint64_t(stage) * (kStageBytes >> 4);
@@ -613,12 +623,10 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
             }
             umma_commit(empty0 + 8 * stage);
           }
-          __syncwarp();
           started |= live;
         }
       }
-      if (lane == 0) umma_commit(tfull0 + 8 * a);
-      __syncwarp();
+      umma_commit(tfull0 + 8 * a);
       if (!ok) mbar_drain(tfull0 + 8 * a, use & 1);
       ++acc_iter;
     }
