@@ -10,7 +10,7 @@ Written from the trellis_sparse_mlx README:
   only; this oracle is the "deliberately naive" form that section describes
   (a dict lookup and a per-voxel loop).
 
-Readings where the pages are silent (each also listed in the design doc):
+Readings where the pages are silent:
 
 * tap order: for K = 3, k = 9 (dx + 1) + 3 (dy + 1) + (dz + 1), x slowest;
   for general odd K the same mixed-radix order with radius K // 2;
