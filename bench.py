@@ -45,8 +45,7 @@ DTYPE_NAME = {"f16": "f16", "bf16": "bf16", "f32": "f32"}
 # dram__bytes_read.sum + dram__bytes_write.sum of one k_conv_tc launch, from the
 # ncu capture summarised in profiles/k_conv_tc_<workload>.md (bytes).  Only
 # workloads captured with the current kernel are listed; others report null.
-NCU_TRAFFIC = {"uniform128": 65.024768e6 + 15.813632e6,
-               "resblock64": 103.662336e6 + 36.518144e6}
+NCU_TRAFFIC: dict = {}
 # fp32 features run on the CUDA cores with fp64 accumulation: the ALU bound is
 # the fp64 FMA rate, 148 SMs x 64 fp64 lanes x 2 FLOP x 1.965 GHz.
 FP64_ALU_TFLOPS = 148 * 64 * 2 * 1.965e9 / 1e12

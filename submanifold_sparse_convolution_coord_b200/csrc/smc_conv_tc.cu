@@ -239,6 +239,7 @@ struct ConvArgs {
   const int32_t* tile_off;    // [n_tiles + 1] first slot of each tile
   const uint32_t* tile_mask;  // [n_tiles] active taps of each tile
   const int32_t* out_row;     // [n_tiles * 128], -1 = padding row
+  const int32_t* group_order; // [n_groups] group of the q-th item, most taps first
   uint32_t* work_counter;     // [0] next item, [1] CTAs finished; both 0 between launches
   int32_t* status;
   int64_t n;
@@ -253,8 +254,9 @@ struct ConvArgs {
 // A work item is a group of G consecutive tiles (in plan order) and one
 // BN-wide block of output channels.  The group's taps are the union of its
 // tiles' taps; a W chunk is loaded once per stage and multiplied into every
-// tile of the group that has that tap.  Items are numbered heaviest first and
-// handed out dynamically, so every SM stays busy until the end.
+// tile of the group that has that tap.  Items are numbered by the tap count of
+// their group, most first (longest-processing-time order), and handed out
+// dynamically, so every SM stays busy until the end.
 template <int G>
 struct Group {
   int w;         // item number, -1 = no more work
@@ -271,7 +273,8 @@ __device__ __forceinline__ Group<G> group_of(const ConvArgs& a, int w) {
   Group<G> gr;
   gr.w = w;
   const int q = w / a.n_blocks;
-  gr.tile0 = (a.n_groups - 1 - q) * G;  // groups with the largest tap sets first
+  // groups with the largest tap sets first; K = 1 items are all alike
+  gr.tile0 = (a.dense ? a.n_groups - 1 - q : a.group_order[q]) * G;
   gr.n0 = (w - q * a.n_blocks) * BN;
   gr.all = 0;
 #pragma unroll
@@ -783,6 +786,8 @@ int launch_cfg(const Plan& plan, bool dense, const void* feats, const void* W, v
   a.tile_off = plan.tile_off;
   a.tile_mask = plan.tile_mask;
   a.out_row = plan.out_row;
+  static_assert(G == 1 || G == 2, "work-item orders exist for one and two tiles per item");
+  a.group_order = plan.group_order[G - 1];
   a.status = plan.status;
   a.n = plan.n;
   a.cin = cin;

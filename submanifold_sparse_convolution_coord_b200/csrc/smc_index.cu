@@ -274,6 +274,25 @@ k_tile_gather(const int32_t* __restrict__ perm, const int32_t* __restrict__ nbr,
   }
 }
 
+// Sort keys of the work-item groups: group g covers tiles g*G .. g*G+G-1; its
+// key is 27 minus the tap count of their union, listed from the last group to
+// the first, so a stable ascending sort yields most taps first and, among
+// equal tap counts, the later (heavier-masked) groups first.
+__global__ void k_group_keys(const uint32_t* __restrict__ tile_mask, int64_t n_tiles, int G,
+                             int64_t n_groups, uint32_t* __restrict__ keys,
+                             int32_t* __restrict__ vals) {
+  const int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+  if (i >= n_groups) return;
+  const int64_t g = n_groups - 1 - i;
+  uint32_t u = 0;
+  for (int k = 0; k < G; ++k) {
+    const int64_t t = g * G + k;
+    if (t < n_tiles) u |= tile_mask[t];
+  }
+  keys[i] = uint32_t(kTaps - __popc(u));
+  vals[i] = int32_t(g);
+}
+
 template <class T>
 int dev_alloc(T** p, size_t count, cudaStream_t s) {
   *p = nullptr;
@@ -311,7 +330,14 @@ struct Scratch {
   uint32_t* hist = nullptr;
   uint32_t* tile_ntaps = nullptr;
   unsigned long long* stats = nullptr;
+  uint32_t* gkeys[2] = {nullptr, nullptr};
+  int32_t* gvals = nullptr;
+  uint32_t* ghist = nullptr;
   void release(cudaStream_t s) {
+    dev_free(gkeys[0], s);
+    dev_free(gkeys[1], s);
+    dev_free(gvals, s);
+    dev_free(ghist, s);
     dev_free(keys, s);
     dev_free(vals, s);
     for (int i = 0; i < 2; ++i) {
@@ -441,6 +467,28 @@ int build_plan_impl(const int32_t* coords, int64_t n, int32_t stride, int64_t ta
                                                     plan->tile_off, plan->tile_taps, plan->gidx,
                                                     plan->out_row);
   SMC_LAUNCHED();
+
+  // 5. work-item order for one and two tiles per item: one stable radix pass
+  // over the (27 - tap count) keys, which are below 256
+  {
+    const int gblocks = int((nt + kSortTile - 1) / kSortTile);
+    SMC_TRY(dev_alloc(&sc.gkeys[0], size_t(nt), s));
+    SMC_TRY(dev_alloc(&sc.gkeys[1], size_t(nt), s));
+    SMC_TRY(dev_alloc(&sc.gvals, size_t(nt), s));
+    SMC_TRY(dev_alloc(&sc.ghist, size_t(256) * gblocks, s));
+    for (int G = 1; G <= 2; ++G) {
+      const int64_t ng = (nt + G - 1) / G;
+      const int nb = int((ng + kSortTile - 1) / kSortTile);
+      SMC_TRY(dev_alloc(&plan->group_order[G - 1], size_t(ng), s));
+      k_group_keys<<<grid_for(ng, 256), 256, 0, s>>>(plan->tile_mask, nt, G, ng, sc.gkeys[0],
+                                                      sc.gvals);
+      k_radix_hist<<<nb, kSortThreads, 0, s>>>(sc.gkeys[0], ng, 0, sc.ghist, nb);
+      k_scan_exclusive<<<1, 1024, 0, s>>>(sc.ghist, int64_t(256) * nb);
+      k_radix_scatter<<<nb, kSortThreads, 0, s>>>(sc.gkeys[0], sc.gvals, sc.gkeys[1],
+                                                  plan->group_order[G - 1], ng, 0, sc.ghist, nb);
+      SMC_LAUNCHED();
+    }
+  }
   if (cudaStreamSynchronize(s) != cudaSuccess) return SMC_ERR_CUDA;
   return SMC_OK;
 }
@@ -459,6 +507,8 @@ void free_plan(Plan* plan) {
   dev_free(plan->out_row, s);
   dev_free(plan->status, s);
   dev_free(plan->work_counter, s);
+  dev_free(plan->group_order[0], s);
+  dev_free(plan->group_order[1], s);
   cudaStreamSynchronize(s);
 }
 

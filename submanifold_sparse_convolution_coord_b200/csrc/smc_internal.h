@@ -37,6 +37,9 @@ struct Plan {
   int32_t* out_row = nullptr;     // [n_tiles * 128] voxel written per plan row, -1 = none
   int32_t* status = nullptr;      // device status word
   uint32_t* work_counter = nullptr;  // tensor-core kernel's item counter (+ finished CTAs)
+  // group_order[G - 1][q]: the q-th work item's group of G consecutive tiles,
+  // most taps first (G = 1, 2), so the largest items are handed out first
+  int32_t* group_order[2] = {nullptr, nullptr};
   int64_t useful_pairs = 0;
   int64_t issued_rows_taps = 0;
 };
