@@ -145,8 +145,10 @@ int smc_build_neighbor_map_static(const int32_t* coords_dev, int64_t n, int32_t 
  *
  * Tensor-core path when cin % 64 == 0 and cout % 64 == 0 (f16/bf16); any
  * other cin, cout >= 1 runs on the CUDA-core kernel.  feats and out must not
- * overlap.  Errors: SMC_ERR_INVALID (null / misaligned pointers, K not 1 or 3,
- * bad dtype, cin or cout < 1), SMC_ERR_CUDA (launch failure).  A device-side
+ * overlap.  The current device must be the one the handle was built on.
+ * Errors: SMC_ERR_INVALID (null / misaligned pointers, K not 1 or 3, bad
+ * dtype, cin or cout < 1, another current device), SMC_ERR_CUDA (launch
+ * failure).  A device-side
  * wait that gives up is reported later by smc_device_status.
  */
 int smc_forward(smc_handle_t h, const void* feats, const void* W, void* out, int K,

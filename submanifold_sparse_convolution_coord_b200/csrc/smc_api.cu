@@ -101,6 +101,11 @@ int smc_build_index(const int32_t* coords_dev, int64_t n, int32_t stride,
 int smc_forward(smc_handle_t h, const void* feats, const void* W, void* out, int K, int cin,
                 int cout, int dtype, smc_stream_t stream) {
   if (!h) return SMC_ERR_INVALID;
+  // the handle's plan lives on the device it was built on; launching from
+  // another current device would hand that device foreign pointers
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess) return SMC_ERR_CUDA;
+  if (cur != h->device) return SMC_ERR_INVALID;
   if (K != 1 && K != 3) return SMC_ERR_INVALID;
   if (elem_bytes(dtype) == 0 || cin < 1 || cout < 1) return SMC_ERR_INVALID;
   const smc::Plan& plan = h->plan;

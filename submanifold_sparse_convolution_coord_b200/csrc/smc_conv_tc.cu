@@ -767,12 +767,18 @@ int launch_cfg(const Plan& plan, bool dense, const void* feats, const void* W, v
   static_assert(kSmem <= 227 * 1024, "shared memory");
   static_assert(threads_for(STAGES, WPS) <= 1024, "threads");
   auto kern = k_conv_tc<BN, BK, STAGES, G, WPS, BF16, NBUF>;
-  static bool attr_set = false;
-  if (!attr_set) {
+  // the shared-memory limit is a per-device function attribute: set it once
+  // on each device this configuration runs on
+  constexpr int kMaxDev = 64;
+  static bool attr_set[kMaxDev] = {};
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SMC_ERR_CUDA;
+  const bool cached = dev >= 0 && dev < kMaxDev && attr_set[dev];
+  if (!cached) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) !=
         cudaSuccess)
       return SMC_ERR_CUDA;
-    attr_set = true;
+    if (dev >= 0 && dev < kMaxDev) attr_set[dev] = true;
   }
   CUtensorMap wmap, fmap;
   const int taps = dense ? 1 : kTaps;
