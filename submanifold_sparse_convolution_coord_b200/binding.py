@@ -116,9 +116,10 @@ def smc_build_index(coords: torch.Tensor, stride: int = 1, table_capacity: int =
     ptr = _dev_ptr(coords, "coords", torch.int32)
     opts = _Options(int(table_capacity), ORDER_CODE[order], 0)
     h = ctypes.c_void_p()
-    rc = lib().smc_build_index_ex(ctypes.c_void_p(ptr), coords.shape[0], int(stride),
-                                  ctypes.byref(opts), _stream(stream, coords.device),
-                                  ctypes.byref(h))
+    with torch.cuda.device(coords.device):  # the handle belongs to the coordinates' device
+        rc = lib().smc_build_index_ex(ctypes.c_void_p(ptr), coords.shape[0], int(stride),
+                                      ctypes.byref(opts), _stream(stream, coords.device),
+                                      ctypes.byref(h))
     _check(rc, "smc_build_index")
     return h.value
 
@@ -131,9 +132,12 @@ def smc_forward(handle: int, feats: torch.Tensor, W: torch.Tensor, out: torch.Te
     fp = _dev_ptr(feats, "feats", dtype)
     wp = _dev_ptr(W, "W", dtype)
     op = _dev_ptr(out, "out", dtype)
-    rc = lib().smc_forward(ctypes.c_void_p(handle), ctypes.c_void_p(fp), ctypes.c_void_p(wp),
-                           ctypes.c_void_p(op), int(K), int(cin), int(cout), DTYPE_CODE[dtype],
-                           _stream(stream, feats.device))
+    if W.device != feats.device or out.device != feats.device:
+        raise ValueError("feats, W and out must be on one device")
+    with torch.cuda.device(feats.device):  # the library checks it is the handle's device
+        rc = lib().smc_forward(ctypes.c_void_p(handle), ctypes.c_void_p(fp), ctypes.c_void_p(wp),
+                               ctypes.c_void_p(op), int(K), int(cin), int(cout),
+                               DTYPE_CODE[dtype], _stream(stream, feats.device))
     _check(rc, "smc_forward")
 
 
