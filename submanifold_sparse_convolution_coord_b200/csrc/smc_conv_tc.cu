@@ -21,14 +21,15 @@
 //               accepts it (about one MMA time), so a single issuer's own
 //               loop and waits between stages would idle the tensor core;
 //               two issuers cover each other's gaps;
-//   warps 2-5   epilogue: tensor memory -> registers -> fp16/bf16 -> global,
-//               overlapping the MMAs of the next work item;
-//   warp 6      scheduler: takes work items (heaviest first) from a global
+//   warps 2-5   epilogue: tensor memory -> registers -> fp16/bf16 -> global;
+//               with two accumulator sets (NBUF = 2) it overlaps the MMAs of
+//               the next work item;
+//   warp 6      scheduler: takes work items (most taps first) from a global
 //               counter and decodes each one's tile masks and slot offsets
 //               into a small shared-memory queue read by every other role;
 //   warps 7..   gather, WPS (4 or 2) warps per pipeline stage slot: warp q of
 //               slot i copies rows 128/WPS q .. of every tile the stage feeds
-//               (64 channels, 128 bytes per row) with 16-byte cp.async
+//               (BK = 64 or 32 channels, 128 or 64 bytes per row) with 16-byte cp.async
 //               (zero-filled for absent neighbours) into a 128-byte-swizzled
 //               K-major tile; each lane's mbarrier arrival fires when its
 //               copies land, so no thread waits on its copies.  Many warps
