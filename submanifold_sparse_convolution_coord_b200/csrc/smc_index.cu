@@ -13,7 +13,11 @@
 //               taps coincide;
 //   4. plan     per tile, the OR of its rows' masks (the taps the tensor-core
 //               kernel multiplies; the others are skipped) and a compact
-//               gather index [tile][active tap][128 rows].
+//               gather index [tile][active tap][128 rows];
+//   5. items    for work items of one and of two consecutive tiles, the
+//               groups in decreasing order of their union's tap count (one
+//               stable radix pass), so the convolution hands out its largest
+//               items first.
 #include <algorithm>
 #include <cstdio>
 #include <cstring>
