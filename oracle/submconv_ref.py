@@ -27,7 +27,7 @@ the tolerance of the half-precision comparison is measured against.
 Pins (tests/test_oracle_pins.py): dense conv3d on a zero-filled grid with
 outputs taken at active sites (brute force), K = 1 equals a Linear layer, an
 isolated voxel gives feats @ W[centre], a hand-worked two-voxel case
-(tests/golden/two_voxel.json) that separates c + d from c - d, and
+(tests/golden/hand_worked.json) that separates c + d from c - d, and
 neighbour-map invariants (centre tap is the voxel itself, symmetry).
 """
 from __future__ import annotations

@@ -7,12 +7,15 @@
   feats @ W[centre], the interior of a dense block of ones gives the sum of
   all weights;
 * the hand-worked fixtures in tests/golden/hand_worked.json, which separate
-  feats[c+d] from feats[c-d] and fix the tap order;
+  feats[c+d] from feats[c-d], fix the tap order, and fix the error scale
+  S = sum |feats[c+d]| |W[d]| (equal to the output when no terms cancel, above
+  |out| in the mixed-sign case);
 * neighbour-map invariants and an O(N^2) brute-force neighbour search;
 * the C++ oracle against the Python one.
 
-Planted mistakes (a flipped offset, a dropped tap, a transposed weight) are
-applied to a copy of the oracle here, on the CPU, to show the pins catch them.
+Planted mistakes (a flipped offset, a dropped tap, a transposed weight; for S:
+absent taps counted, a product of sums, |out| in place of S) are applied to a
+copy of the oracle here, on the CPU, to show the pins catch them.
 """
 import json
 import os
@@ -108,16 +111,44 @@ def _golden_cases():
         return json.load(fh)["cases"]
 
 
+def _golden_weights(case) -> np.ndarray:
+    """W[k] = k + 1, or (-1)^k (k + 1) for the 'alternating' cases (Cin = Cout = 1)."""
+    k = np.arange(27, dtype=np.float64)
+    w = k + 1.0
+    if case.get("weights") == "alternating":
+        w = np.where(k % 2 == 0, 1.0, -1.0) * w
+    return w.reshape(27, 1, 1)
+
+
 @pytest.mark.parametrize("case", _golden_cases(), ids=lambda c: c["name"])
 def test_hand_worked_golden(case):
+    """Output and error scale S of both oracles equal the hand-worked values
+    (exactly: every product and sum is a small integer)."""
     coords = np.array(case["coords"], np.int32)
     feats = np.array(case["feats"], np.float64)[:, None]
-    W = (np.arange(27, dtype=np.float64) + 1.0).reshape(27, 1, 1)
-    out, _ = ref.submconv(coords, feats, W)
+    W = _golden_weights(case)
+    out, scale = ref.submconv(coords, feats, W)
     assert out[:, 0].tolist() == case["expected"]
+    assert scale[:, 0].tolist() == case["expected_scale"]
     nbr = native.neighbor_map(coords)
-    out_c = native.submconv(feats, W, nbr, want_scale=False)
+    out_c, scale_c = native.submconv(feats, W, nbr)
     assert out_c[:, 0].tolist() == case["expected"]
+    assert scale_c[:, 0].tolist() == case["expected_scale"]
+
+
+def test_scale_bounds_and_reaches_output():
+    """S >= |out| always (triangle inequality), with equality exactly when no
+    terms cancel: all-positive inputs give S == out, element by element."""
+    rng = np.random.default_rng(13)
+    coords = _random_sites(rng, 8, 2, 0.3)
+    feats = rng.standard_normal((len(coords), 4))
+    W = rng.standard_normal((27, 4, 3))
+    out, scale = ref.submconv(coords, feats, W)
+    assert np.all(scale >= np.abs(out) - 1e-12)
+    assert np.any(scale > np.abs(out) + 1e-6)  # random signs do cancel somewhere
+    out_p, scale_p = ref.submconv(coords, np.abs(feats), np.abs(W))
+    np.testing.assert_allclose(scale_p, out_p, rtol=1e-13, atol=0)
+    np.testing.assert_allclose(scale_p, scale, rtol=1e-13, atol=0)  # S depends on |f|, |W| only
 
 
 def test_map_invariants_and_bruteforce_search():
@@ -216,9 +247,10 @@ def test_planted_mistakes_are_caught(mutation):
     for case in _golden_cases():
         coords = np.array(case["coords"], np.int32)
         feats = np.array(case["feats"])[:, None]
-        W = (np.arange(27, dtype=np.float64) + 1.0).reshape(27, 1, 1)
+        W = _golden_weights(case)
         if _mutant_submconv(coords, feats, W, mutation)[:, 0].tolist() != case["expected"]:
             caught = True
+        assert _mutant_submconv(coords, feats, W, "none")[:, 0].tolist() == case["expected"]
     rng = np.random.default_rng(12)
     coords = _random_sites(rng, 8, 1, 0.5)
     feats = rng.standard_normal((len(coords), 3))
@@ -228,4 +260,41 @@ def test_planted_mistakes_are_caught(mutation):
         caught = True
     # the unmutated form agrees with brute force
     assert np.allclose(_mutant_submconv(coords, feats, W, "none"), dense, rtol=1e-9, atol=1e-9)
+    assert caught
+
+
+def _mutant_scale(coords, feats, W, mutation):
+    """The error scale S with a planted mistake."""
+    nbr = ref.neighbor_map(coords)
+    f = np.abs(np.asarray(feats, np.float64))
+    w = np.abs(np.asarray(W, np.float64))
+    n = len(f)
+    S = np.zeros((n, w.shape[2]))
+    for i in range(n):
+        for k in range(27):
+            j = nbr[i, k]
+            if mutation == "all_taps":  # absent neighbours counted with the voxel's own row
+                S[i] += f[j if j >= 0 else i] @ w[k]
+            elif j >= 0:
+                S[i] += f[j] @ w[k]
+    if mutation == "product_of_sums":  # (sum |f|) * (sum |W|) over the active taps
+        for i in range(n):
+            ks = [k for k in range(27) if nbr[i, k] >= 0]
+            S[i] = f[nbr[i, ks]].sum(axis=0) @ w[ks].sum(axis=0)
+    if mutation == "abs_of_sum":  # |out| instead of sum |f| |W|
+        S = np.abs(ref.submconv(coords, feats, W)[0])
+    return S
+
+
+@pytest.mark.parametrize("mutation", ["all_taps", "product_of_sums", "abs_of_sum"])
+def test_planted_scale_mistakes_are_caught(mutation):
+    caught = False
+    for case in _golden_cases():
+        coords = np.array(case["coords"], np.int32)
+        feats = np.array(case["feats"])[:, None]
+        W = _golden_weights(case)
+        if _mutant_scale(coords, feats, W, mutation)[:, 0].tolist() != case["expected_scale"]:
+            caught = True
+        # the unmutated form reproduces the hand-worked values
+        assert _mutant_scale(coords, feats, W, "none")[:, 0].tolist() == case["expected_scale"]
     assert caught
