@@ -42,9 +42,9 @@ PAGES_CONV_MS = 13.8  # M3 Ultra, same layer (trellis_sparse_mlx README, "Perfor
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 DTYPE_NAME = {"f16": "f16", "bf16": "bf16", "f32": "f32"}
-# dram__bytes_read.sum + dram__bytes_write.sum of one k_conv_tc launch, from the
-# ncu capture summarised in profiles/k_conv_tc_<workload>.md (bytes).  Only
-# workloads captured with the current kernel are listed; others report null.
+# dram__bytes_read.sum + dram__bytes_write.sum of one convolution launch of the
+# current kernel, per (workload, layer), from an ncu capture of that launch
+# (bytes).  Workloads not captured with the current kernel report null.
 NCU_TRAFFIC: dict = {}
 # fp32 features run on the CUDA cores with fp64 accumulation: the ALU bound is
 # the fp64 FMA rate, 148 SMs x 64 fp64 lanes x 2 FLOP x 1.965 GHz.
@@ -123,10 +123,19 @@ def useful_flops(pairs: int, cin: int, cout: int) -> float:
     return 2.0 * pairs * cin * cout
 
 
-def conv_bytes(n: int, cin: int, cout: int, elem: int, slots: int) -> int:
+def conv_bytes(n: int, cin: int, cout: int, elem: int, slots: int, K: int = 3) -> int:
     """Algorithmic HBM bytes of one conv launch: feature rows read once, output
-    rows written once, the compact gather index read once, W read once."""
-    return n * cin * elem + n * cout * elem + slots * 128 * 4 + 27 * cin * cout * elem
+    rows written once, the compact gather index read once (K = 3 only), W read
+    once."""
+    idx = slots * 128 * 4 if K == 3 else 0
+    return n * cin * elem + n * cout * elem + idx + K ** 3 * cin * cout * elem
+
+
+OCCUPANCY = {
+    "bernoulli": "each cell active independently with p = 0.10",
+    "exact": "exactly 10% of cells, uniform, drawn without replacement",
+    "shells": "2-voxel-thick shells of the union of 8 random ellipsoids",
+}
 
 
 def index_build_bytes(n: int, slots: int) -> int:
@@ -182,7 +191,12 @@ def reduce_max_sum(value_max: float, value_sum: float, world: int, device) -> tu
 # ----------------------------------------------------------------------------
 # CPU oracle timing (reference arm and cpu_baseline)
 # ----------------------------------------------------------------------------
-def time_oracle(inp, budget_s: float, seed: int = 0, cache: dict | None = None) -> dict:
+def time_oracle(inp, budget_s: float, seed: int = 0, cache: dict | None = None,
+                layer: int = 0, feats_in: torch.Tensor | None = None) -> dict:
+    """The C++ oracle on the host cores over a random row sample of one layer
+    sized to about budget_s seconds (the dict and neighbour map are built over
+    all voxels).  feats_in is the layer's input when it is not the workload's
+    first layer."""
     from oracle import native
     t = {}
     if cache is not None and "nbr" in cache:
@@ -191,8 +205,10 @@ def time_oracle(inp, budget_s: float, seed: int = 0, cache: dict | None = None) 
         nbr = native.neighbor_map(inp.coords, 3, 1, timings=t)
         if cache is not None:
             cache["nbr"], cache["t"] = nbr, dict(t)
-    w = inp.weights[0]
-    feats = inp.feats.double().numpy()
+    if inp.workload.layers[layer].K == 1:
+        nbr = np.arange(inp.n, dtype=np.int32)[:, None]
+    w = inp.weights[layer]
+    feats = (inp.feats if feats_in is None else feats_in).double().numpy()
     W = w.double().numpy()
     cin, cout = W.shape[1], W.shape[2]
     pairs_per_row = (nbr >= 0).sum(axis=1)
@@ -270,13 +286,15 @@ def run_ours(args) -> None:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
     binding.lib()
-    inp = synth.make_inputs(args.workload, n_layers=1)
-    w = inp.workload
-    layer = w.layers[0]
-    cin, cout = layer.cin, layer.cout
+    w = synth.WORKLOADS[args.workload]
+    if not 0 <= args.layer < len(w.layers):
+        raise ValueError(f"{args.workload} has {len(w.layers)} layer(s)")
+    inp = synth.make_inputs(args.workload, n_layers=args.layer + 1)
+    layer = w.layers[args.layer]
+    K, cin, cout = layer.K, layer.cin, layer.cout
     coords = torch.from_numpy(inp.coords).to(dev)
     feats = inp.feats.to(dev)
-    W = inp.weights[0].to(dev)
+    W = inp.weights[args.layer].to(dev)
     out = torch.empty((inp.n, cout), dtype=feats.dtype, device=dev)
     elem = feats.element_size()
     stream = torch.cuda.current_stream(dev)
@@ -292,14 +310,25 @@ def run_ours(args) -> None:
         build_ms.append((time.perf_counter() - t0) * 1e3)
         idx.close()
     idx = binding.SubMIndex(coords)
-    pairs, issued = idx.plan_stats()
+    pairs3, issued3 = idx.plan_stats()
+    slots = issued3 // 128
+    # a later layer's input is what the earlier layers of the block produce
+    for li in range(args.layer):
+        lw = w.layers[li]
+        nxt = torch.empty((inp.n, lw.cout), dtype=feats.dtype, device=dev)
+        binding.smc_forward(idx.handle, feats, inp.weights[li].to(dev), nxt, lw.K, lw.cin, lw.cout)
+        feats = nxt
+    torch.cuda.synchronize()
+    if K == 3:
+        pairs, issued = pairs3, issued3
+    else:  # 1x1x1: every voxel is its own single pair; rows run in 128-row tiles
+        pairs, issued = inp.n, idx.n_tiles * 128
     flops = useful_flops(pairs, cin, cout)
-    slots = issued // 128
 
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
 
     def step():
-        binding.smc_forward(idx.handle, feats, W, out, 3, cin, cout)
+        binding.smc_forward(idx.handle, feats, W, out, K, cin, cout)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -333,15 +362,15 @@ def run_ours(args) -> None:
         raise RuntimeError("device status word set during the timed region")
 
     # ---- end to end through the C ABI with host buffers ----
-    feats_h = inp.feats.pin_memory()
-    W_h = inp.weights[0].pin_memory()
+    feats_h = feats.cpu().pin_memory()
+    W_h = inp.weights[args.layer].pin_memory()
     out_h = torch.empty((inp.n, cout), dtype=feats.dtype).pin_memory()
     e2e_steps = max(3, min(args.steps, 50))
 
     def e2e_step():
         feats.copy_(feats_h, non_blocking=True)
         W.copy_(W_h, non_blocking=True)
-        binding.smc_forward(idx.handle, feats, W, out, 3, cin, cout)
+        binding.smc_forward(idx.handle, feats, W, out, K, cin, cout)
         out_h.copy_(out, non_blocking=True)
 
     for _ in range(3):
@@ -361,7 +390,7 @@ def run_ours(args) -> None:
     peaks, peak_kind = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     achieved = flops / (conv_ms * 1e-3) / 1e12
-    algo_bytes = conv_bytes(inp.n, cin, cout, elem, slots)
+    algo_bytes = conv_bytes(inp.n, cin, cout, elem, slots, K)
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
 
     line = {
@@ -374,8 +403,8 @@ def run_ours(args) -> None:
                         if args.workload == "uniform128" else None),
         "dtype": DTYPE_NAME[w.dtype], "data": "synthetic",
         "config": {"workload": args.workload, "grid": w.grid, "batch": w.batch,
-                   "n_voxels": inp.n, "cin": cin, "cout": cout, "K": 3,
-                   "occupancy": "exactly 10% of cells, uniform", "seed": 0,
+                   "n_voxels": inp.n, "layer": args.layer, "cin": cin, "cout": cout, "K": K,
+                   "occupancy": OCCUPANCY[w.sparsity], "seed": 0,
                    "l2": "flushed between steps (256 MB write, outside the timed events)",
                    "parallelism": f"replicas x{world}"},
         "conv_ms": conv_ms_max,
@@ -387,7 +416,7 @@ def run_ours(args) -> None:
         "roofline": {"bound": "tensor" if w.dtype != "f32" else "alu", "achieved": achieved,
                      "peak": peak if w.dtype != "f32" else FP64_ALU_TFLOPS, "unit": "TFLOP/s",
                      "frac": achieved / (peak if w.dtype != "f32" else FP64_ALU_TFLOPS),
-                     "traffic": NCU_TRAFFIC.get(args.workload),
+                     "traffic": NCU_TRAFFIC.get((args.workload, args.layer)),
                      "peak_source": (f"bf16 dense burst, {peak_kind} (fp16 assumed equal)"
                                      if w.dtype != "f32" else
                                      "fp64 FMA: 148 SMs x 64 lanes x 2 x 1.965 GHz"),
@@ -402,7 +431,8 @@ def run_ours(args) -> None:
         "timed_wall_s": wall_s,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        ob = time_oracle(inp, budget_s=args.cpu_budget)
+        ob = time_oracle(inp, budget_s=args.cpu_budget, layer=args.layer,
+                         feats_in=feats.cpu() if args.layer > 0 else None)
         line["cpu_baseline"] = {
             "value": ob["tflops"], "unit": "TFLOP/s", "cores": ob["cores"], "kind": "oracle",
             "sample": (f"{args.workload}: oracle dict + neighbour map over all {ob['n']} voxels "
@@ -422,6 +452,9 @@ def main(argv=None) -> None:
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="uniform128", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--layer", type=int, default=0,
+                    help="layer of the workload to time (resblock64: 0 = 3x3x3 512->512, "
+                         "1 = 1x1x1 512->1024)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     args = ap.parse_args(argv)

@@ -21,8 +21,13 @@
  *   - "device pointer" = memory of the current CUDA device, contiguous,
  *     row-major, at least 16-byte aligned.  The caller owns every pointer it
  *     passes; the library never frees or retains them past the call.
- *   - Every function returns an smc_status (0 = SMC_OK) unless noted; on an
- *     error nothing has been launched and output buffers are untouched.
+ *   - Every function returns an smc_status (0 = SMC_OK) unless noted.  Errors
+ *     found in the arguments are reported before anything is launched and
+ *     leave every output buffer untouched.  Errors only the device can see
+ *     (duplicate coordinates, out-of-range coordinates, a full hash table)
+ *     are reported after the kernels that found them have run: the index
+ *     build then frees what it allocated and writes no caller buffer, and
+ *     smc_build_neighbor_map_static leaves map_dev undefined.
  *   - No call falls back to the CPU.  There is no alternative backend.
  */
 #ifndef SMC_H_
@@ -61,16 +66,30 @@ enum smc_order {
   SMC_ORDER_INPUT = 1  /* rows in input order (ablation) */
 };
 
+/* How neighbours are looked up (smc_index_options.lookup); both give the same
+ * map, bit for bit. */
+enum smc_lookup {
+  SMC_LOOKUP_HASH = 0, /* open-addressing hash of packed coordinates: default */
+  SMC_LOOKUP_SORT = 1  /* packed 64-bit keys radix-sorted, binary search per tap
+                          ("Running TRELLIS.2 on a Mac (3/3)", "E. Vectorizing mesh
+                          extraction": pack into int64, sort, searchsorted) */
+};
+
 typedef struct smc_index_options {
   int64_t table_capacity; /* hash slots; 0 = smallest power of two >= 2N.  A
                              value < N makes the build fail with
                              SMC_ERR_TABLE_FULL (used to test that path). */
   int32_t order;          /* enum smc_order */
-  int32_t reserved;       /* must be 0 */
+  int32_t lookup;         /* enum smc_lookup */
 } smc_index_options;
 
 /*
- * Build the neighbour map and the tile plan of a coordinate set.
+ * Build the neighbour map and the tile plan of a coordinate set: the
+ * "prepared device gather index" of the trellis_sparse_mlx README
+ * ("Performance": caching it, not only the raw indice map, is what made the
+ * layer compute-bound; "What's in it": a SparseTensor is coords [N,4] +
+ * feats [N,C] with an indice-map cache).  Build once per coordinate set, then
+ * run any number of smc_forward calls on the handle.
  *
  * coords_dev : device pointer, int32 [n][4] = (b, x, y, z), any row order.
  * n          : number of voxels, >= 0 (n == 0 gives an empty handle).
@@ -111,12 +130,16 @@ int smc_build_index_ex(const int32_t* coords_dev, int64_t n, int32_t stride,
  * map_dev    : device pointer, int32 [n][27], written like
  *              smc_get_neighbor_map's output (-1 = no active neighbour).
  * stream     : the work is queued on this stream, which the call then
- *              synchronises to read the status word.
+ *              synchronises to read the status word.  After
+ *              SMC_ERR_DUPLICATE or SMC_ERR_RANGE the kernels have run and
+ *              map_dev holds undefined values.
  *
  * Scratch: the coordinate hash table lives in one fixed array of static
- * device memory (about 14 MiB), reserved on every GPU that loads libsmc and
+ * device memory (about 18 MiB), reserved on every GPU that loads libsmc and
  * held until the process exits.  The first call on a device looks up that
- * array's device address; make that first call before any stream capture.
+ * array's device address (looked up again only if the device's CUDA context
+ * changes, e.g. after cudaDeviceReset); make that first call before any
+ * stream capture.
  * Every call, from any stream or host thread, uses the same array and clears
  * the part it needs first, so calls that overlap on the GPU race with each
  * other and must be serialised by the caller.
@@ -126,7 +149,10 @@ int smc_build_neighbor_map_static(const int32_t* coords_dev, int64_t n, int32_t 
                                   int32_t* map_dev, smc_stream_t stream);
 
 /*
- * SubMConv3d forward over the handle's voxels.
+ * SubMConv3d forward over the handle's voxels (trellis_sparse_mlx README,
+ * "What's in it": the submanifold 3x3x3 and 1x1x1 sparse convolution;
+ * "Correctness": feats[c+d] is gathered, cross-correlation).  Implements the
+ * sum written at the top of this file.
  *
  * feats : device pointer, [n][cin] of dtype.
  * W     : device pointer, [K^3][cin][cout] of dtype, W[k][ci][co] (tap k as
@@ -154,11 +180,103 @@ int smc_build_neighbor_map_static(const int32_t* coords_dev, int64_t n, int32_t 
 int smc_forward(smc_handle_t h, const void* feats, const void* W, void* out, int K,
                 int cin, int cout, int dtype, smc_stream_t stream);
 
+/*
+ * Input gradient of smc_forward ("Metal-native replacement for flex_gemm
+ * bottleneck?", "Fixed" / "Open": the bwd-input pass next to fwd):
+ *
+ *     grad_in[j] = sum over (i, k) with voxel j at coords[i] + stride*d(k)
+ *                  of grad_out[i] @ W[k]^T
+ *
+ * the adjoint of the forward sum in feats.  Because j is i's tap-k neighbour
+ * exactly when i is j's tap-(26 - k) neighbour, this is the forward
+ * convolution of grad_out with the weights W'[k] = W[26 - k]^T, and it runs on
+ * the same kernels and tile plan.
+ *
+ * grad_out : device pointer, [n][cout] of dtype.
+ * W        : device pointer, [K^3][cin][cout] of dtype (the forward weights).
+ * grad_in  : device pointer, [n][cin] of dtype; every element is overwritten.
+ * K, cin, cout, dtype, stream: as for smc_forward (cin and cout are the
+ *         forward layer's).  Asynchronous; calls on one handle must be
+ *         stream-ordered.  The transposed weights live in a workspace the
+ *         handle owns, allocated stream-ordered (cudaMallocAsync) the first
+ *         time a call needs more than it holds.
+ * Errors: as smc_forward, plus SMC_ERR_OOM.
+ */
+int smc_backward_input(smc_handle_t h, const void* grad_out, const void* W, void* grad_in, int K,
+                       int cin, int cout, int dtype, smc_stream_t stream);
+
+/*
+ * Weight gradient of smc_forward (the bwd-weight pass of the same passage):
+ *
+ *     dW[k] = sum over voxels i with an active tap-k neighbour j
+ *             of outer(feats[j], grad_out[i])          ([cin][cout] per tap)
+ *
+ * feats    : device pointer, [n][cin] of dtype (the forward input).
+ * grad_out : device pointer, [n][cout] of dtype.
+ * dW       : device pointer, float32 [K^3][cin][cout]; every element is
+ *            overwritten (taps with no pair get zeros).  fp32 whatever dtype
+ *            is: weight gradients are accumulated in fp32 (f16/bf16 inputs,
+ *            tensor cores) or fp64 (f32 inputs, CUDA cores) and rounded once.
+ * The sum over pairs is split over CTAs; the partial sums go to a workspace
+ * the handle owns (allocated stream-ordered when it must grow) and are added
+ * in a fixed order, so the result is deterministic.  Asynchronous; calls on
+ * one handle must be stream-ordered.
+ * Errors: as smc_forward, plus SMC_ERR_OOM.
+ */
+int smc_backward_weight(smc_handle_t h, const void* feats, const void* grad_out, float* dW, int K,
+                        int cin, int cout, int dtype, smc_stream_t stream);
+
+/*
+ * x2 downsample of a sparse tensor by maximum (trellis_sparse_mlx README,
+ * "What's in it": the downsample half of the subdivide / downsample row, "x2
+ * max-pool", reduce="amax").  The parent of (b, x, y, z) is
+ * (b, x >> 1, y >> 1, z >> 1); every parent appears once, in lexicographic
+ * (b, x, y, z) order, and its row is the element-wise maximum of its
+ * children's rows (an exact copy of one input value per element).
+ *
+ * coords_dev     : device pointer, int32 [n][4], any order, no duplicates
+ *                  needed (duplicates simply share a parent).
+ * feats_dev      : device pointer, [n][c] of dtype.
+ * out_coords_dev : device pointer, int32 [n][4] (room for n parents).
+ * out_feats_dev  : device pointer, [n][c] of dtype.
+ * out_n          : host pointer, receives the number of parents m; rows
+ *                  [0, m) of both outputs are written.
+ * Queued on stream, which the call synchronises to read m back; its scratch
+ * is allocated and freed stream-ordered (cudaMallocAsync).
+ * Errors: SMC_ERR_INVALID, _RANGE (coordinates outside the packing limits;
+ * outputs undefined), _OOM, _CUDA, _UNSUPPORTED (n >= 2^31).
+ */
+int smc_downsample2(const int32_t* coords_dev, int64_t n, const void* feats_dev, int c, int dtype,
+                    int32_t* out_coords_dev, void* out_feats_dev, int64_t* out_n,
+                    smc_stream_t stream);
+
+/*
+ * x2 subdivision (the subdivide half of the same row, "x2 coord expansion"):
+ * voxel i's 8 children (b, 2x + dx, 2y + dy, 2z + dz) are rows 8 i + c,
+ * c = 4 dx + 2 dy + dz, and each carries a copy of voxel i's row.
+ *
+ * coords_dev     : device pointer, int32 [n][4]; x, y, z must be below 32768
+ *                  so the children stay inside the packing limits.
+ * feats_dev      : device pointer, [n][c] of dtype.
+ * out_coords_dev : device pointer, int32 [8 n][4].
+ * out_feats_dev  : device pointer, [8 n][c] of dtype.
+ * Synchronises stream to read the range check.  Errors: SMC_ERR_INVALID,
+ * _RANGE (outputs undefined), _OOM, _CUDA, _UNSUPPORTED (n >= 2^28).
+ */
+int smc_subdivide2(const int32_t* coords_dev, int64_t n, const void* feats_dev, int c, int dtype,
+                   int32_t* out_coords_dev, void* out_feats_dev, smc_stream_t stream);
+
 /* Copy the int32 [n][27] neighbour map (-1 = no active neighbour) into
- * map_dev, asynchronously on stream. */
+ * map_dev, asynchronously on stream.  Entry [i][k] is the row j whose
+ * coordinates are coords[i] + stride * d(k) in the same batch: the indice map
+ * of the trellis_sparse_mlx README ("What's in it", SparseTensor's indice-map
+ * cache), with -1 in place of its unnamed sentinel ("Performance"). */
 int smc_get_neighbor_map(smc_handle_t h, int32_t* map_dev, smc_stream_t stream);
 
-/* Host-side counts fixed at build time: useful_pairs = number of
+/* Work counts of the tile plan (the masked implicit GEMM skips every tap no
+ * row of a 128-row tile uses, as mtlgemm's sorted_idx / valid_kernel masking
+ * does in "Metal-native replacement for flex_gemm bottleneck?", "Fixed").
+ * Host-side counts fixed at build time: useful_pairs = number of
  * (voxel, active neighbour) pairs, i.e. non-sentinel map entries;
  * issued_rows_taps = rows x taps the tensor-core kernel multiplies for K = 3
  * (128 rows per tile times the taps active anywhere in the tile).  Either
@@ -179,7 +297,9 @@ int smc_get_tile_plan(smc_handle_t h, int32_t* perm_dev, uint32_t* tile_mask_dev
  * SMC_OK, or SMC_ERR_TIMEOUT when a kernel gave up waiting. */
 int smc_device_status(smc_handle_t h, smc_stream_t stream);
 
-/* Release the handle's device memory (synchronous).  NULL is ignored. */
+/* Release the handle's device memory.  Synchronous: it first waits for all
+ * work queued on the handle's device, on every stream, so a forward still in
+ * flight never reads freed memory.  NULL is ignored. */
 void smc_destroy(smc_handle_t h);
 
 /* Static string for a status code. */

@@ -40,6 +40,10 @@ def load():
     lib.oracle_neighbor_map.restype = ctypes.c_int
     lib.oracle_submconv.argtypes = [p, p, p, i64, i32, i32, i32, p, i64, p, p, p]
     lib.oracle_submconv.restype = ctypes.c_int
+    lib.oracle_submconv_backward_input.argtypes = [p, p, p, i64, i32, i32, i32, p, p, p]
+    lib.oracle_submconv_backward_input.restype = ctypes.c_int
+    lib.oracle_submconv_backward_weight.argtypes = [p, p, p, i64, i32, i32, i32, p, p, p]
+    lib.oracle_submconv_backward_weight.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -99,3 +103,53 @@ def submconv(feats, W, nbr, rows=None, want_scale: bool = True,
     if timings is not None:
         timings["conv_ms"] = t_conv.value
     return (out, scale) if want_scale else out
+
+
+def submconv_backward_input(grad_out, W, nbr, want_scale: bool = True,
+                            timings: dict | None = None):
+    """Input gradient float64 [N, Cin] (and its error scale) of the
+    convolution with weights W [taps, Cin, Cout] over the neighbour map nbr."""
+    lib = load()
+    g = np.ascontiguousarray(grad_out, dtype=np.float64)
+    w = np.ascontiguousarray(W, dtype=np.float64)
+    m = np.ascontiguousarray(nbr, dtype=np.int32)
+    n, cout = g.shape
+    taps, cin, wcout = w.shape
+    if wcout != cout or m.shape != (n, taps):
+        raise ValueError("shape mismatch")
+    gin = np.empty((n, cin), dtype=np.float64)
+    scale = np.empty((n, cin), dtype=np.float64) if want_scale else None
+    t = ctypes.c_double(0.0)
+    rc = lib.oracle_submconv_backward_input(_ptr(g), _ptr(w), _ptr(m), n, taps, cin, cout,
+                                            _ptr(gin), _ptr(scale) if want_scale else None,
+                                            ctypes.byref(t))
+    if rc != 0:
+        raise ValueError(f"oracle_submconv_backward_input failed ({rc})")
+    if timings is not None:
+        timings["bwd_input_ms"] = t.value
+    return (gin, scale) if want_scale else gin
+
+
+def submconv_backward_weight(feats, grad_out, nbr, want_scale: bool = True,
+                             timings: dict | None = None):
+    """Weight gradient float64 [taps, Cin, Cout] (and its error scale)."""
+    lib = load()
+    f = np.ascontiguousarray(feats, dtype=np.float64)
+    g = np.ascontiguousarray(grad_out, dtype=np.float64)
+    m = np.ascontiguousarray(nbr, dtype=np.int32)
+    n, cin = f.shape
+    gn, cout = g.shape
+    taps = m.shape[1]
+    if gn != n or m.shape[0] != n:
+        raise ValueError("shape mismatch")
+    dW = np.empty((taps, cin, cout), dtype=np.float64)
+    scale = np.empty((taps, cin, cout), dtype=np.float64) if want_scale else None
+    t = ctypes.c_double(0.0)
+    rc = lib.oracle_submconv_backward_weight(_ptr(f), _ptr(g), _ptr(m), n, taps, cin, cout,
+                                             _ptr(dW), _ptr(scale) if want_scale else None,
+                                             ctypes.byref(t))
+    if rc != 0:
+        raise ValueError(f"oracle_submconv_backward_weight failed ({rc})")
+    if timings is not None:
+        timings["bwd_weight_ms"] = t.value
+    return (dW, scale) if want_scale else dW

@@ -149,4 +149,93 @@ int oracle_submconv(const double* feats, const double* W, const int32_t* nbr, in
   return bad ? -1 : 0;
 }
 
+// Input gradient (the adjoint of oracle_submconv in feats): every forward
+// term feats[j] @ W[k] added to out[i] (j = nbr[i, k]) sends W[k] @ grad_out[i]
+// back to row j.  The (i, k) pairs of each row j are listed first (i, then k,
+// ascending), then every row j sums its own list, so the result does not
+// depend on the thread count.  grad_out: double [n, cout]; gin / scale:
+// double [n, cin]; scale (may be nullptr) is the same sum over |W| |grad_out|.
+int oracle_submconv_backward_input(const double* grad_out, const double* W, const int32_t* nbr,
+                                   int64_t n, int32_t taps, int32_t cin, int32_t cout,
+                                   double* gin, double* scale, double* ms) {
+  if (n < 0 || taps < 1 || cin < 1 || cout < 1) return -1;
+  auto t0 = std::chrono::steady_clock::now();
+  std::vector<int64_t> start(size_t(n) + 1, 0);
+  for (int64_t i = 0; i < n * taps; ++i) {
+    const int64_t j = nbr[i];
+    if (j >= n) return -1;
+    if (j >= 0) ++start[size_t(j) + 1];
+  }
+  for (int64_t j = 0; j < n; ++j) start[size_t(j) + 1] += start[size_t(j)];
+  std::vector<int64_t> list(size_t(start[size_t(n)]));  // entries i * taps + k
+  std::vector<int64_t> fill(start.begin(), start.end() - 1);
+  for (int64_t e = 0; e < n * taps; ++e) {
+    const int64_t j = nbr[e];
+    if (j >= 0) list[size_t(fill[size_t(j)]++)] = e;
+  }
+#pragma omp parallel for schedule(dynamic, 64)
+  for (int64_t j = 0; j < n; ++j) {
+    double* acc = gin + j * cin;
+    double* mag = scale ? scale + j * cin : nullptr;
+    for (int32_t ci = 0; ci < cin; ++ci) acc[ci] = 0.0;
+    if (mag)
+      for (int32_t ci = 0; ci < cin; ++ci) mag[ci] = 0.0;
+    for (int64_t e = start[size_t(j)]; e < start[size_t(j) + 1]; ++e) {
+      const int64_t i = list[size_t(e)] / taps, k = list[size_t(e)] % taps;
+      const double* g = grad_out + i * cout;
+      const double* w = W + k * cin * cout;
+      for (int32_t ci = 0; ci < cin; ++ci) {
+        const double* wr = w + int64_t(ci) * cout;
+        double s = 0.0, m = 0.0;
+        for (int32_t co = 0; co < cout; ++co) {
+          s += wr[co] * g[co];
+          if (mag) m += std::fabs(wr[co]) * std::fabs(g[co]);
+        }
+        acc[ci] += s;
+        if (mag) mag[ci] += m;
+      }
+    }
+  }
+  if (ms) *ms = ms_since(t0);
+  return 0;
+}
+
+// Weight gradient (the adjoint of oracle_submconv in W): dW[k] is the sum
+// over voxels i with a neighbour j = nbr[i, k] of outer(feats[j], grad_out[i]),
+// voxels in ascending order.  feats: double [n, cin]; grad_out: double
+// [n, cout]; dW / scale: double [taps, cin, cout] (scale may be nullptr).
+int oracle_submconv_backward_weight(const double* feats, const double* grad_out,
+                                    const int32_t* nbr, int64_t n, int32_t taps, int32_t cin,
+                                    int32_t cout, double* dW, double* scale, double* ms) {
+  if (n < 0 || taps < 1 || cin < 1 || cout < 1) return -1;
+  auto t0 = std::chrono::steady_clock::now();
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+  for (int64_t kc = 0; kc < int64_t(taps) * cin; ++kc) {
+    const int64_t k = kc / cin, ci = kc % cin;
+    double* acc = dW + kc * cout;
+    double* mag = scale ? scale + kc * cout : nullptr;
+    for (int32_t co = 0; co < cout; ++co) acc[co] = 0.0;
+    if (mag)
+      for (int32_t co = 0; co < cout; ++co) mag[co] = 0.0;
+    for (int64_t i = 0; i < n; ++i) {
+      const int64_t j = nbr[i * taps + k];
+      if (j < 0) continue;
+      if (j >= n) {
+        bad = 1;
+        continue;
+      }
+      const double fv = feats[j * cin + ci];
+      const double* g = grad_out + i * cout;
+      for (int32_t co = 0; co < cout; ++co) acc[co] += fv * g[co];
+      if (mag) {
+        const double af = std::fabs(fv);
+        for (int32_t co = 0; co < cout; ++co) mag[co] += af * std::fabs(g[co]);
+      }
+    }
+  }
+  if (ms) *ms = ms_since(t0);
+  return bad ? -1 : 0;
+}
+
 }  // extern "C"

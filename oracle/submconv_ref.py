@@ -100,3 +100,97 @@ def submconv(coords, feats, W, K: int = 3, stride: int = 1, nbr=None):
         out[i] = acc
         scale[i] = mag
     return out, scale
+
+
+# ----------------------------------------------------------------------------
+# Backward passes ("Metal-native replacement for flex_gemm bottleneck?",
+# "Fixed" / "Open": fwd / bwd-input / bwd-weight, each with its own parity).
+# The forward map is linear in feats and in W; these are its two adjoints,
+# written straight from the forward sum: every term feats[j] @ W[k] that the
+# forward adds to out[i] (j = nbr[i, k]) sends grad_out[i] @ W[k]^T back to
+# feats[j] and outer(feats[j], grad_out[i]) to W[k].
+# ----------------------------------------------------------------------------
+def submconv_backward_input(coords, grad_out, W, K: int = 3, stride: int = 1, nbr=None):
+    """grad_feats float64 [N, Cin] and its error scale (the same sum over
+    |grad_out[i]| @ |W[k]|^T), for loss gradient grad_out [N, Cout]."""
+    g = np.asarray(grad_out, dtype=np.float64)
+    w = np.asarray(W, dtype=np.float64)
+    if nbr is None:
+        nbr = neighbor_map(coords, K, stride)
+    n, cin = g.shape[0], w.shape[1]
+    gin = np.zeros((n, cin), dtype=np.float64)
+    scale = np.zeros((n, cin), dtype=np.float64)
+    aw = np.abs(w)
+    for i in range(n):
+        for k in range(K ** 3):
+            j = nbr[i, k]
+            if j < 0:
+                continue
+            gin[j] += w[k] @ g[i]
+            scale[j] += aw[k] @ np.abs(g[i])
+    return gin, scale
+
+
+def submconv_backward_weight(coords, feats, grad_out, K: int = 3, stride: int = 1, nbr=None):
+    """dW float64 [K^3, Cin, Cout] and its error scale (the same sum of
+    outer(|feats[j]|, |grad_out[i]|))."""
+    f = np.asarray(feats, dtype=np.float64)
+    g = np.asarray(grad_out, dtype=np.float64)
+    if nbr is None:
+        nbr = neighbor_map(coords, K, stride)
+    taps = K ** 3
+    dW = np.zeros((taps, f.shape[1], g.shape[1]), dtype=np.float64)
+    scale = np.zeros_like(dW)
+    for i in range(f.shape[0]):
+        for k in range(taps):
+            j = nbr[i, k]
+            if j < 0:
+                continue
+            dW[k] += np.outer(f[j], g[i])
+            scale[k] += np.outer(np.abs(f[j]), np.abs(g[i]))
+    return dW, scale
+
+
+# ----------------------------------------------------------------------------
+# x2 coordinate ops (trellis_sparse_mlx README, "What's in it": subdivide /
+# downsample -- x2 coordinate expansion; x2 max-pool, upstream passing
+# reduce="amax" although its docstring says "average").
+# Readings: the parent of (b, x, y, z) is (b, x // 2, y // 2, z // 2); the
+# downsampled tensor lists each parent once, in lexicographic (b, x, y, z)
+# order (batch-contiguous, like every SparseTensor here), with the element-wise
+# maximum of its children's rows; subdivision gives every voxel its 8 children
+# (b, 2x + dx, 2y + dy, 2z + dz), child c = 4 dx + 2 dy + dz, parents in input
+# order, each child carrying its parent's row.
+# ----------------------------------------------------------------------------
+def downsample2(coords, feats):
+    """(parent coords int32 [M, 4], float64 feats [M, C]) of the x2 max-pool."""
+    f = np.asarray(feats, dtype=np.float64)
+    groups = {}
+    for i, (b, x, y, z) in enumerate(np.asarray(coords).tolist()):
+        groups.setdefault((b, x // 2, y // 2, z // 2), []).append(i)
+    keys = sorted(groups)
+    out_c = np.array(keys, dtype=np.int32).reshape(-1, 4)
+    out_f = np.zeros((len(keys), f.shape[1]), dtype=np.float64)
+    for p, key in enumerate(keys):
+        rows = groups[key]
+        acc = f[rows[0]].copy()
+        for r in rows[1:]:
+            acc = np.maximum(acc, f[r])
+        out_f[p] = acc
+    return out_c, out_f
+
+
+def subdivide2(coords, feats):
+    """(child coords int32 [8N, 4], float64 feats [8N, C]) of the x2 expansion."""
+    f = np.asarray(feats, dtype=np.float64)
+    rows = np.asarray(coords).tolist()
+    out_c = np.zeros((8 * len(rows), 4), dtype=np.int32)
+    out_f = np.zeros((8 * len(rows), f.shape[1]), dtype=np.float64)
+    for i, (b, x, y, z) in enumerate(rows):
+        for dx in (0, 1):
+            for dy in (0, 1):
+                for dz in (0, 1):
+                    c = 8 * i + 4 * dx + 2 * dy + dz
+                    out_c[c] = (b, 2 * x + dx, 2 * y + dy, 2 * z + dz)
+                    out_f[c] = f[i]
+    return out_c, out_f

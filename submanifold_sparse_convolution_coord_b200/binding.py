@@ -25,12 +25,14 @@ STATUS = {
 }
 DTYPE_CODE = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
 ORDER_CODE = {"mask": 0, "input": 1}
+LOOKUP_CODE = {"hash": 0, "sort": 1}
 
 # every symbol include/smc.h declares
 EXPORTS = (
     "smc_build_index", "smc_build_index_ex", "smc_forward", "smc_get_neighbor_map",
     "smc_get_plan_stats", "smc_get_sizes", "smc_get_tile_plan", "smc_device_status",
     "smc_destroy", "smc_status_string", "smc_version", "smc_build_neighbor_map_static",
+    "smc_backward_input", "smc_backward_weight", "smc_downsample2", "smc_subdivide2",
 )
 
 
@@ -42,7 +44,7 @@ class SmcError(RuntimeError):
 
 class _Options(ctypes.Structure):
     _fields_ = [("table_capacity", ctypes.c_int64), ("order", ctypes.c_int32),
-                ("reserved", ctypes.c_int32)]
+                ("lookup", ctypes.c_int32)]
 
 
 _lib = None
@@ -62,6 +64,10 @@ def lib() -> ctypes.CDLL:
     L.smc_build_index.argtypes = [p, i64, i32, ctypes.POINTER(p)]
     L.smc_build_index_ex.argtypes = [p, i64, i32, ctypes.POINTER(_Options), p, ctypes.POINTER(p)]
     L.smc_forward.argtypes = [p, p, p, p, i, i, i, i, p]
+    L.smc_backward_input.argtypes = [p, p, p, p, i, i, i, i, p]
+    L.smc_backward_weight.argtypes = [p, p, p, p, i, i, i, i, p]
+    L.smc_downsample2.argtypes = [p, i64, p, i, i, p, p, ctypes.POINTER(i64), p]
+    L.smc_subdivide2.argtypes = [p, i64, p, i, i, p, p, p]
     L.smc_get_neighbor_map.argtypes = [p, p, p]
     L.smc_get_plan_stats.argtypes = [p, ctypes.POINTER(i64), ctypes.POINTER(i64)]
     L.smc_get_sizes.argtypes = [p, ctypes.POINTER(i64), ctypes.POINTER(i64)]
@@ -109,12 +115,13 @@ def _dev_ptr(t: torch.Tensor, name: str, dtype=None) -> int:
 # same-name wrappers
 # ----------------------------------------------------------------------------
 def smc_build_index(coords: torch.Tensor, stride: int = 1, table_capacity: int = 0,
-                    order: str = "mask", stream: Optional[torch.cuda.Stream] = None) -> int:
+                    order: str = "mask", stream: Optional[torch.cuda.Stream] = None,
+                    lookup: str = "hash") -> int:
     """coords: CUDA int32 [N, 4] (b, x, y, z).  Returns the raw handle (int)."""
     if coords.dim() != 2 or coords.shape[1] != 4:
         raise ValueError("coords must be [N, 4]")
     ptr = _dev_ptr(coords, "coords", torch.int32)
-    opts = _Options(int(table_capacity), ORDER_CODE[order], 0)
+    opts = _Options(int(table_capacity), ORDER_CODE[order], LOOKUP_CODE[lookup])
     h = ctypes.c_void_p()
     with torch.cuda.device(coords.device):  # the handle belongs to the coordinates' device
         rc = lib().smc_build_index_ex(ctypes.c_void_p(ptr), coords.shape[0], int(stride),
@@ -139,6 +146,78 @@ def smc_forward(handle: int, feats: torch.Tensor, W: torch.Tensor, out: torch.Te
                                ctypes.c_void_p(op), int(K), int(cin), int(cout),
                                DTYPE_CODE[dtype], _stream(stream, feats.device))
     _check(rc, "smc_forward")
+
+
+def smc_backward_input(handle: int, grad_out: torch.Tensor, W: torch.Tensor,
+                       grad_in: torch.Tensor, K: int, cin: int, cout: int,
+                       stream: Optional[torch.cuda.Stream] = None) -> None:
+    dtype = grad_out.dtype
+    if dtype not in DTYPE_CODE:
+        raise ValueError(f"unsupported dtype {dtype}")
+    gp = _dev_ptr(grad_out, "grad_out", dtype)
+    wp = _dev_ptr(W, "W", dtype)
+    ip = _dev_ptr(grad_in, "grad_in", dtype)
+    with torch.cuda.device(grad_out.device):
+        rc = lib().smc_backward_input(ctypes.c_void_p(handle), ctypes.c_void_p(gp),
+                                      ctypes.c_void_p(wp), ctypes.c_void_p(ip), int(K), int(cin),
+                                      int(cout), DTYPE_CODE[dtype], _stream(stream, grad_out.device))
+    _check(rc, "smc_backward_input")
+
+
+def smc_backward_weight(handle: int, feats: torch.Tensor, grad_out: torch.Tensor,
+                        dW: torch.Tensor, K: int, cin: int, cout: int,
+                        stream: Optional[torch.cuda.Stream] = None) -> None:
+    dtype = feats.dtype
+    if dtype not in DTYPE_CODE:
+        raise ValueError(f"unsupported dtype {dtype}")
+    fp = _dev_ptr(feats, "feats", dtype)
+    gp = _dev_ptr(grad_out, "grad_out", dtype)
+    wp = _dev_ptr(dW, "dW", torch.float32)
+    with torch.cuda.device(feats.device):
+        rc = lib().smc_backward_weight(ctypes.c_void_p(handle), ctypes.c_void_p(fp),
+                                       ctypes.c_void_p(gp), ctypes.c_void_p(wp), int(K), int(cin),
+                                       int(cout), DTYPE_CODE[dtype], _stream(stream, feats.device))
+    _check(rc, "smc_backward_weight")
+
+
+def smc_downsample2(coords: torch.Tensor, feats: torch.Tensor,
+                    stream: Optional[torch.cuda.Stream] = None) -> tuple:
+    """x2 downsample by maximum: (parent coords int32 [M, 4], feats [M, C])."""
+    if coords.dim() != 2 or coords.shape[1] != 4 or feats.dim() != 2 or \
+            feats.shape[0] != coords.shape[0]:
+        raise ValueError("coords must be [N, 4] and feats [N, C]")
+    n, c = feats.shape
+    cp = _dev_ptr(coords, "coords", torch.int32)
+    fp = _dev_ptr(feats, "feats", feats.dtype)
+    out_c = torch.empty((max(n, 1), 4), dtype=torch.int32, device=coords.device)
+    out_f = torch.empty((max(n, 1), c), dtype=feats.dtype, device=coords.device)
+    m = ctypes.c_int64(0)
+    with torch.cuda.device(coords.device):
+        rc = lib().smc_downsample2(ctypes.c_void_p(cp), n, ctypes.c_void_p(fp), int(c),
+                                   DTYPE_CODE[feats.dtype], ctypes.c_void_p(out_c.data_ptr()),
+                                   ctypes.c_void_p(out_f.data_ptr()), ctypes.byref(m),
+                                   _stream(stream, coords.device))
+    _check(rc, "smc_downsample2")
+    return out_c[:m.value], out_f[:m.value]
+
+
+def smc_subdivide2(coords: torch.Tensor, feats: torch.Tensor,
+                   stream: Optional[torch.cuda.Stream] = None) -> tuple:
+    """x2 subdivision: (child coords int32 [8N, 4], feats [8N, C])."""
+    if coords.dim() != 2 or coords.shape[1] != 4 or feats.dim() != 2 or \
+            feats.shape[0] != coords.shape[0]:
+        raise ValueError("coords must be [N, 4] and feats [N, C]")
+    n, c = feats.shape
+    cp = _dev_ptr(coords, "coords", torch.int32)
+    fp = _dev_ptr(feats, "feats", feats.dtype)
+    out_c = torch.empty((max(8 * n, 1), 4), dtype=torch.int32, device=coords.device)
+    out_f = torch.empty((max(8 * n, 1), c), dtype=feats.dtype, device=coords.device)
+    with torch.cuda.device(coords.device):
+        rc = lib().smc_subdivide2(ctypes.c_void_p(cp), n, ctypes.c_void_p(fp), int(c),
+                                  DTYPE_CODE[feats.dtype], ctypes.c_void_p(out_c.data_ptr()),
+                                  ctypes.c_void_p(out_f.data_ptr()), _stream(stream, coords.device))
+    _check(rc, "smc_subdivide2")
+    return out_c[:8 * n], out_f[:8 * n]
 
 
 def smc_get_neighbor_map(handle: int, map_out: torch.Tensor,
@@ -195,9 +274,9 @@ class SubMIndex:
     (the cached indice map of the README's SparseTensor)."""
 
     def __init__(self, coords: torch.Tensor, stride: int = 1, table_capacity: int = 0,
-                 order: str = "mask"):
+                 order: str = "mask", lookup: str = "hash"):
         self.device = coords.device
-        self.handle = smc_build_index(coords, stride, table_capacity, order)
+        self.handle = smc_build_index(coords, stride, table_capacity, order, lookup=lookup)
         self.n, self.n_tiles = smc_get_sizes(self.handle)
 
     def close(self) -> None:
@@ -244,6 +323,30 @@ class SubMIndex:
         if out is None:
             out = torch.empty((self.n, cout), dtype=feats.dtype, device=feats.device)
         smc_forward(self.handle, feats, W, out, K, cin, cout)
+        return out
+
+
+    def backward_input(self, grad_out: torch.Tensor, W: torch.Tensor, K: int = 3,
+                       out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """Gradient of the forward with respect to feats, [N, Cin]."""
+        taps, cin, cout = W.shape
+        if taps != K ** 3 or grad_out.dim() != 2 or grad_out.shape != (self.n, cout):
+            raise ValueError("grad_out must be [N, Cout] and W [K^3, Cin, Cout]")
+        if out is None:
+            out = torch.empty((self.n, cin), dtype=grad_out.dtype, device=grad_out.device)
+        smc_backward_input(self.handle, grad_out, W, out, K, cin, cout)
+        return out
+
+    def backward_weight(self, feats: torch.Tensor, grad_out: torch.Tensor, K: int = 3,
+                        out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """Gradient of the forward with respect to W, float32 [K^3, Cin, Cout]."""
+        if feats.dim() != 2 or grad_out.dim() != 2 or feats.shape[0] != self.n or \
+                grad_out.shape[0] != self.n:
+            raise ValueError("feats must be [N, Cin] and grad_out [N, Cout]")
+        cin, cout = feats.shape[1], grad_out.shape[1]
+        if out is None:
+            out = torch.empty((K ** 3, cin, cout), dtype=torch.float32, device=feats.device)
+        smc_backward_weight(self.handle, feats, grad_out, out, K, cin, cout)
         return out
 
 

@@ -10,6 +10,10 @@ struct smc_index {
   int device = 0;
   int32_t stride = 1;
   smc::Plan plan;
+  // workspace of the backward passes (transposed weights, partial sums),
+  // grown stream-ordered; calls on one handle are stream-ordered
+  void* work = nullptr;
+  size_t work_bytes = 0;
 };
 
 namespace {
@@ -26,6 +30,42 @@ int elem_bytes(int dtype) {
     default:
       return 0;
   }
+}
+
+// Make the handle's workspace at least `bytes` long, stream-ordered on s.
+int ensure_workspace(smc_index* h, size_t bytes, cudaStream_t s) {
+  if (bytes <= h->work_bytes) return SMC_OK;
+  if (h->work) cudaFreeAsync(h->work, s);
+  h->work = nullptr;
+  h->work_bytes = 0;
+  bytes = (bytes + 255) & ~size_t(255);
+  if (cudaMallocAsync(&h->work, bytes, s) != cudaSuccess) {
+    cudaGetLastError();
+    h->work = nullptr;
+    return SMC_ERR_OOM;
+  }
+  h->work_bytes = bytes;
+  return SMC_OK;
+}
+
+// Checks shared by the forward and backward calls.
+int check_call(smc_index* h, int K, int cin, int cout, int dtype) {
+  if (!h) return SMC_ERR_INVALID;
+  // the handle's plan lives on the device it was built on; launching from
+  // another current device would hand that device foreign pointers
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess) return SMC_ERR_CUDA;
+  if (cur != h->device) return SMC_ERR_INVALID;
+  if (K != 1 && K != 3) return SMC_ERR_INVALID;
+  if (elem_bytes(dtype) == 0 || cin < 1 || cout < 1) return SMC_ERR_INVALID;
+  return SMC_OK;
+}
+
+int conv(const smc::Plan& plan, bool dense, const void* x, const void* W, void* y, int cin,
+         int cout, int dtype, cudaStream_t s) {
+  if (smc::conv_tc_supported(cin, cout, dtype))
+    return smc::launch_conv_tc(plan, dense, x, W, y, cin, cout, dtype, s);
+  return smc::launch_conv_simt(plan, dense, x, W, y, cin, cout, dtype, s);
 }
 
 }  // namespace
@@ -68,13 +108,15 @@ int smc_build_index_ex(const int32_t* coords_dev, int64_t n, int32_t stride,
   if (n > 0 && !aligned16(coords_dev)) return SMC_ERR_INVALID;
   if (n >= (int64_t(1) << 31) / smc::kTaps) return SMC_ERR_UNSUPPORTED;
   int64_t cap = 0;
-  int32_t order = SMC_ORDER_MASK;
+  int32_t order = SMC_ORDER_MASK, lookup = SMC_LOOKUP_HASH;
   if (opts) {
-    if (opts->reserved != 0 || opts->table_capacity < 0 ||
-        (opts->order != SMC_ORDER_MASK && opts->order != SMC_ORDER_INPUT))
+    if (opts->table_capacity < 0 ||
+        (opts->order != SMC_ORDER_MASK && opts->order != SMC_ORDER_INPUT) ||
+        (opts->lookup != SMC_LOOKUP_HASH && opts->lookup != SMC_LOOKUP_SORT))
       return SMC_ERR_INVALID;
     cap = opts->table_capacity;
     order = opts->order;
+    lookup = opts->lookup;
   }
   smc_index* h = new (std::nothrow) smc_index();
   if (!h) return SMC_ERR_OOM;
@@ -83,7 +125,7 @@ int smc_build_index_ex(const int32_t* coords_dev, int64_t n, int32_t stride,
     return SMC_ERR_CUDA;
   }
   h->stride = stride;
-  const int rc = smc::build_plan(coords_dev, n, stride, cap, order,
+  const int rc = smc::build_plan(coords_dev, n, stride, cap, order, lookup,
                                  reinterpret_cast<cudaStream_t>(stream), &h->plan);
   if (rc != SMC_OK) {
     delete h;
@@ -100,23 +142,72 @@ int smc_build_index(const int32_t* coords_dev, int64_t n, int32_t stride,
 
 int smc_forward(smc_handle_t h, const void* feats, const void* W, void* out, int K, int cin,
                 int cout, int dtype, smc_stream_t stream) {
-  if (!h) return SMC_ERR_INVALID;
-  // the handle's plan lives on the device it was built on; launching from
-  // another current device would hand that device foreign pointers
-  int cur = -1;
-  if (cudaGetDevice(&cur) != cudaSuccess) return SMC_ERR_CUDA;
-  if (cur != h->device) return SMC_ERR_INVALID;
-  if (K != 1 && K != 3) return SMC_ERR_INVALID;
-  if (elem_bytes(dtype) == 0 || cin < 1 || cout < 1) return SMC_ERR_INVALID;
+  const int rc = check_call(h, K, cin, cout, dtype);
+  if (rc != SMC_OK) return rc;
   const smc::Plan& plan = h->plan;
   if (plan.n == 0) return SMC_OK;
   if (!feats || !W || !out) return SMC_ERR_INVALID;
   if (!aligned16(feats) || !aligned16(W) || !aligned16(out)) return SMC_ERR_INVALID;
-  const bool dense = (K == 1);
+  return conv(plan, K == 1, feats, W, out, cin, cout, dtype,
+              reinterpret_cast<cudaStream_t>(stream));
+}
+
+int smc_backward_input(smc_handle_t h, const void* grad_out, const void* W, void* grad_in, int K,
+                       int cin, int cout, int dtype, smc_stream_t stream) {
+  int rc = check_call(h, K, cin, cout, dtype);
+  if (rc != SMC_OK) return rc;
+  const smc::Plan& plan = h->plan;
+  if (plan.n == 0) return SMC_OK;
+  if (!grad_out || !W || !grad_in) return SMC_ERR_INVALID;
+  if (!aligned16(grad_out) || !aligned16(W) || !aligned16(grad_in)) return SMC_ERR_INVALID;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (smc::conv_tc_supported(cin, cout, dtype))
-    return smc::launch_conv_tc(plan, dense, feats, W, out, cin, cout, dtype, s);
-  return smc::launch_conv_simt(plan, dense, feats, W, out, cin, cout, dtype, s);
+  const int taps = K * K * K;
+  rc = ensure_workspace(h, size_t(taps) * cin * cout * elem_bytes(dtype), s);
+  if (rc != SMC_OK) return rc;
+  // grad_in = conv(grad_out, W'), W'[k] = W[taps - 1 - k]^T: [taps][cout][cin]
+  rc = smc::launch_weight_transpose(W, h->work, taps, cin, cout, dtype, s);
+  if (rc != SMC_OK) return rc;
+  return conv(plan, K == 1, grad_out, h->work, grad_in, cout, cin, dtype, s);
+}
+
+int smc_backward_weight(smc_handle_t h, const void* feats, const void* grad_out, float* dW, int K,
+                        int cin, int cout, int dtype, smc_stream_t stream) {
+  int rc = check_call(h, K, cin, cout, dtype);
+  if (rc != SMC_OK) return rc;
+  if (!dW || !aligned16(dW)) return SMC_ERR_INVALID;
+  const smc::Plan& plan = h->plan;
+  if (plan.n > 0 && (!feats || !grad_out || !aligned16(feats) || !aligned16(grad_out)))
+    return SMC_ERR_INVALID;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool dense = (K == 1);
+  rc = ensure_workspace(h, smc::bwd_weight_workspace_bytes(plan, dense, cin, cout, dtype), s);
+  if (rc != SMC_OK) return rc;
+  return smc::launch_bwd_weight(plan, dense, feats, grad_out, dW, cin, cout, dtype, h->work,
+                                smc::wait_limit_ns(), s);
+}
+
+int smc_downsample2(const int32_t* coords_dev, int64_t n, const void* feats_dev, int c, int dtype,
+                    int32_t* out_coords_dev, void* out_feats_dev, int64_t* out_n,
+                    smc_stream_t stream) {
+  if (!out_n || n < 0 || c < 1 || elem_bytes(dtype) == 0) return SMC_ERR_INVALID;
+  *out_n = 0;
+  if (n == 0) return SMC_OK;
+  if (!coords_dev || !feats_dev || !out_coords_dev || !out_feats_dev) return SMC_ERR_INVALID;
+  if (!aligned16(coords_dev) || !aligned16(out_coords_dev)) return SMC_ERR_INVALID;
+  if (n >= (int64_t(1) << 31)) return SMC_ERR_UNSUPPORTED;
+  return smc::downsample2(coords_dev, n, feats_dev, c, dtype, out_coords_dev, out_feats_dev, out_n,
+                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+int smc_subdivide2(const int32_t* coords_dev, int64_t n, const void* feats_dev, int c, int dtype,
+                   int32_t* out_coords_dev, void* out_feats_dev, smc_stream_t stream) {
+  if (n < 0 || c < 1 || elem_bytes(dtype) == 0) return SMC_ERR_INVALID;
+  if (n == 0) return SMC_OK;
+  if (!coords_dev || !feats_dev || !out_coords_dev || !out_feats_dev) return SMC_ERR_INVALID;
+  if (!aligned16(coords_dev) || !aligned16(out_coords_dev)) return SMC_ERR_INVALID;
+  if (n >= (int64_t(1) << 28)) return SMC_ERR_UNSUPPORTED;
+  return smc::subdivide2(coords_dev, n, feats_dev, c, dtype, out_coords_dev, out_feats_dev,
+                         reinterpret_cast<cudaStream_t>(stream));
 }
 
 int smc_get_neighbor_map(smc_handle_t h, int32_t* map_dev, smc_stream_t stream) {
@@ -177,7 +268,11 @@ void smc_destroy(smc_handle_t h) {
   int cur = 0;
   cudaGetDevice(&cur);
   if (cur != h->device) cudaSetDevice(h->device);
-  smc::free_plan(&h->plan);
+  smc::free_plan(&h->plan);  // waits for the device first
+  if (h->work) {
+    cudaFreeAsync(h->work, nullptr);
+    cudaStreamSynchronize(nullptr);
+  }
   if (cur != h->device) cudaSetDevice(cur);
   delete h;
 }

@@ -17,7 +17,9 @@
 //   5. items    for work items of one and of two consecutive tiles, the
 //               groups in decreasing order of their union's tap count (one
 //               stable radix pass), so the convolution hands out its largest
-//               items first.
+//               items first, each written as a 16-byte record (first tile,
+//               tap masks, first gather-index slot) the convolution's
+//               scheduler reads with one load.
 #include <algorithm>
 #include <cstdio>
 #include <cstring>
@@ -28,6 +30,14 @@ namespace smc {
 namespace {
 
 constexpr uint64_t kEmptyKey = ~0ull;
+
+// One open-addressing slot: the packed key and the row it maps to, 16 bytes,
+// so a probe is a single load.  An empty slot holds kEmptyKey.
+struct __align__(16) Slot {
+  unsigned long long key;
+  int32_t val;
+  int32_t pad;
+};
 
 // SplitMix64 output mixer (Steele, Lea and Flood, "Fast splittable
 // pseudorandom number generators", OOPSLA 2014).
@@ -43,8 +53,8 @@ __device__ __forceinline__ uint64_t pack_key(int64_t b, int64_t x, int64_t y, in
 
 __device__ __forceinline__ bool axis_ok(int64_t v) { return v >= 0 && v < kMaxAxis; }
 
-__global__ void k_insert(const int4* __restrict__ coords, int64_t n, uint64_t* keys,
-                         int32_t* vals, uint64_t cap_mask, int32_t* status) {
+__global__ void k_insert(const int4* __restrict__ coords, int64_t n, Slot* table,
+                         uint64_t cap_mask, int32_t* status) {
   const int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
   if (i >= n) return;
   const int4 c = coords[i];
@@ -55,11 +65,10 @@ __global__ void k_insert(const int4* __restrict__ coords, int64_t n, uint64_t* k
   const uint64_t key = pack_key(c.x, c.y, c.z, c.w);
   uint64_t slot = mix64(key) & cap_mask;
   for (uint64_t probe = 0; probe <= cap_mask; ++probe) {
-    const unsigned long long prev = atomicCAS(reinterpret_cast<unsigned long long*>(keys + slot),
-                                              (unsigned long long)kEmptyKey,
-                                              (unsigned long long)key);
+    const unsigned long long prev =
+        atomicCAS(&table[slot].key, (unsigned long long)kEmptyKey, (unsigned long long)key);
     if (prev == kEmptyKey) {
-      vals[slot] = int32_t(i);
+      table[slot].val = int32_t(i);
       return;
     }
     if (prev == key) {
@@ -78,8 +87,8 @@ constexpr int kNbrThreads = kNbrVoxels * kTaps;  // 864
 
 __global__ void __launch_bounds__(kNbrThreads)
 k_neighbors(const int4* __restrict__ coords, int64_t n, int32_t stride,
-            const uint64_t* __restrict__ keys, const int32_t* __restrict__ vals,
-            uint64_t cap_mask, int32_t* __restrict__ nbr, uint32_t* __restrict__ mask) {
+            const Slot* __restrict__ table, uint64_t cap_mask, int32_t* __restrict__ nbr,
+            uint32_t* __restrict__ mask) {
   __shared__ uint32_t smask[kNbrVoxels];
   if (threadIdx.x < kNbrVoxels) smask[threadIdx.x] = 0;
   __syncthreads();
@@ -96,14 +105,80 @@ k_neighbors(const int4* __restrict__ coords, int64_t n, int32_t stride,
       const uint64_t key = pack_key(c.x, x, y, z);
       uint64_t slot = mix64(key) & cap_mask;
       for (uint64_t probe = 0; probe <= cap_mask; ++probe) {
-        const uint64_t kk = keys[slot];
-        if (kk == key) {
-          found = vals[slot];
+        const Slot e = table[slot];
+        if (e.key == key) {
+          found = e.val;
           break;
         }
-        if (kk == kEmptyKey) break;
+        if (e.key == kEmptyKey) break;
         slot = (slot + 1) & cap_mask;
       }
+    }
+    nbr[i * kTaps + k] = found;
+    if (found >= 0) atomicOr(&smask[local], 1u << k);
+  }
+  __syncthreads();
+  if (threadIdx.x < kNbrVoxels) {
+    const int64_t ii = blockIdx.x * int64_t(kNbrVoxels) + threadIdx.x;
+    if (ii < n) mask[ii] = smask[threadIdx.x];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Sort-based lookup (the alternative to the hash): coordinates packed
+// injectively into one 64-bit key, the (key, row) pairs radix-sorted, and
+// every neighbour found by binary search over the sorted keys -- the
+// pack-into-int64 + sort + searchsorted vectorisation of "Running TRELLIS.2 on
+// a Mac (3/3)", section "E. Vectorizing mesh extraction".
+// ---------------------------------------------------------------------------
+__global__ void k_pack_keys(const int4* __restrict__ coords, int64_t n,
+                            unsigned long long* __restrict__ keys, int32_t* __restrict__ vals,
+                            int32_t* status) {
+  const int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+  if (i >= n) return;
+  const int4 c = coords[i];
+  if (c.x < 0 || c.x >= kMaxBatch || !axis_ok(c.y) || !axis_ok(c.z) || !axis_ok(c.w)) {
+    atomicOr(status, kDevRange);
+    keys[i] = ~0ull - uint64_t(i);  // unique, above every valid key: matches nothing
+  } else {
+    keys[i] = pack_key(c.x, c.y, c.z, c.w);
+  }
+  vals[i] = int32_t(i);
+}
+
+__global__ void k_sorted_dups(const unsigned long long* __restrict__ keys, int64_t n,
+                              int32_t* status) {
+  const int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+  if (i >= 1 && i < n && keys[i] == keys[i - 1]) atomicOr(status, kDevDuplicate);
+}
+
+__global__ void __launch_bounds__(kNbrThreads)
+k_neighbors_sorted(const int4* __restrict__ coords, int64_t n, int32_t stride,
+                   const unsigned long long* __restrict__ skeys, const int32_t* __restrict__ svals,
+                   int32_t* __restrict__ nbr, uint32_t* __restrict__ mask) {
+  __shared__ uint32_t smask[kNbrVoxels];
+  if (threadIdx.x < kNbrVoxels) smask[threadIdx.x] = 0;
+  __syncthreads();
+  const int local = threadIdx.x / kTaps;
+  const int k = threadIdx.x - local * kTaps;
+  const int64_t i = blockIdx.x * int64_t(kNbrVoxels) + local;
+  if (i < n) {
+    const int4 c = coords[i];
+    const int64_t x = int64_t(c.y) + int64_t(stride) * (k / 9 - 1);
+    const int64_t y = int64_t(c.z) + int64_t(stride) * ((k / 3) % 3 - 1);
+    const int64_t z = int64_t(c.w) + int64_t(stride) * (k % 3 - 1);
+    int32_t found = -1;
+    if (axis_ok(x) && axis_ok(y) && axis_ok(z)) {
+      const unsigned long long key = pack_key(c.x, x, y, z);
+      int64_t lo = 0, hi = n;  // first position with skeys[pos] >= key
+      while (lo < hi) {
+        const int64_t mid = (lo + hi) >> 1;
+        if (skeys[mid] < key)
+          lo = mid + 1;
+        else
+          hi = mid;
+      }
+      if (lo < n && skeys[lo] == key) found = svals[lo];
     }
     nbr[i * kTaps + k] = found;
     if (found >= 0) atomicOr(&smask[local], 1u << k);
@@ -139,93 +214,6 @@ __global__ void k_iota(int32_t* out, int64_t n) {
   if (i < n) out[i] = int32_t(i);
 }
 
-// ---------------------------------------------------------------------------
-// Stable LSD radix sort, 8 bits per pass: per-block digit histograms, one
-// exclusive scan in (digit, block) order, then a stable scatter that ranks
-// equal digits inside a block in index order.
-// ---------------------------------------------------------------------------
-constexpr int kSortThreads = 256;
-constexpr int kSortRounds = 16;
-constexpr int kSortTile = kSortThreads * kSortRounds;  // 4096 items per block
-
-__global__ void __launch_bounds__(kSortThreads)
-k_radix_hist(const uint32_t* __restrict__ keys, int64_t n, int shift, uint32_t* hist,
-             int nblocks) {
-  __shared__ uint32_t h[256];
-  h[threadIdx.x] = 0;
-  __syncthreads();
-  const int64_t base = blockIdx.x * int64_t(kSortTile);
-  for (int j = 0; j < kSortRounds; ++j) {
-    const int64_t idx = base + j * kSortThreads + threadIdx.x;
-    if (idx < n) atomicAdd(&h[(keys[idx] >> shift) & 255u], 1u);
-  }
-  __syncthreads();
-  hist[int64_t(threadIdx.x) * nblocks + blockIdx.x] = h[threadIdx.x];
-}
-
-// In-place exclusive scan of m 32-bit counts by one block of 1024 threads.
-__global__ void __launch_bounds__(1024) k_scan_exclusive(uint32_t* data, int64_t m) {
-  __shared__ uint32_t part[1024];
-  const int64_t per = (m + 1023) / 1024;
-  const int64_t lo = std::min<int64_t>(threadIdx.x * per, m);
-  const int64_t hi = std::min<int64_t>(lo + per, m);
-  uint32_t s = 0;
-  for (int64_t i = lo; i < hi; ++i) s += data[i];
-  part[threadIdx.x] = s;
-  __syncthreads();
-  for (int off = 1; off < 1024; off <<= 1) {
-    const uint32_t v = threadIdx.x >= unsigned(off) ? part[threadIdx.x - off] : 0u;
-    __syncthreads();
-    part[threadIdx.x] += v;
-    __syncthreads();
-  }
-  uint32_t run = threadIdx.x ? part[threadIdx.x - 1] : 0u;
-  for (int64_t i = lo; i < hi; ++i) {
-    const uint32_t v = data[i];
-    data[i] = run;
-    run += v;
-  }
-}
-
-__global__ void __launch_bounds__(kSortThreads)
-k_radix_scatter(const uint32_t* __restrict__ keys_in, const int32_t* __restrict__ vals_in,
-                uint32_t* __restrict__ keys_out, int32_t* __restrict__ vals_out, int64_t n,
-                int shift, const uint32_t* __restrict__ offsets, int nblocks) {
-  constexpr int kWarps = kSortThreads / 32;
-  __shared__ uint32_t run[256];
-  __shared__ uint32_t wcnt[kWarps][256];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  run[tid] = offsets[int64_t(tid) * nblocks + blockIdx.x];
-  for (int w = 0; w < kWarps; ++w) wcnt[w][tid] = 0;
-  __syncthreads();
-  const int64_t base = blockIdx.x * int64_t(kSortTile);
-  for (int j = 0; j < kSortRounds; ++j) {
-    const int64_t idx = base + j * kSortThreads + tid;
-    const bool valid = idx < n;
-    const uint32_t key = valid ? keys_in[idx] : 0u;
-    const int32_t val = valid ? vals_in[idx] : 0;
-    const uint32_t d = valid ? ((key >> shift) & 255u) : (256u + lane);  // invalid lanes never match
-    const uint32_t peers = __match_any_sync(0xffffffffu, d);
-    const uint32_t rank = __popc(peers & ((1u << lane) - 1u));
-    if (valid && rank == 0) wcnt[warp][d] = __popc(peers);
-    __syncthreads();
-    if (valid) {
-      uint32_t pos = run[d] + rank;
-      for (int w = 0; w < warp; ++w) pos += wcnt[w][d];
-      keys_out[pos] = key;
-      vals_out[pos] = val;
-    }
-    __syncthreads();
-    uint32_t tot = 0;
-    for (int w = 0; w < kWarps; ++w) {
-      tot += wcnt[w][tid];
-      wcnt[w][tid] = 0;
-    }
-    run[tid] += tot;
-    __syncthreads();
-  }
-}
-
 // One block of 128 threads per tile: OR of the rows' masks, its tap count,
 // and the two plan counters (useful pairs, issued rows x taps).
 __global__ void __launch_bounds__(kTileRows)
@@ -255,13 +243,12 @@ k_tile_mask(const int32_t* __restrict__ perm, const uint32_t* __restrict__ mask,
   }
 }
 
-// One block of 128 threads per tile: the tile's tap list and, for each active
-// tap, the voxel each plan row gathers (or -1).
+// One block of 128 threads per tile: for each active tap of the tile, the
+// voxel each plan row gathers (or -1), and the voxel each row writes.
 __global__ void __launch_bounds__(kTileRows)
 k_tile_gather(const int32_t* __restrict__ perm, const int32_t* __restrict__ nbr, int64_t n,
               const uint32_t* __restrict__ tile_mask, const int32_t* __restrict__ tile_off,
-              uint8_t* __restrict__ tile_taps, int32_t* __restrict__ gidx,
-              int32_t* __restrict__ out_row) {
+              int32_t* __restrict__ gidx, int32_t* __restrict__ out_row) {
   const int64_t tile = blockIdx.x;
   const int64_t p = tile * kTileRows + threadIdx.x;
   const int32_t v = p < n ? perm[p] : -1;
@@ -272,7 +259,6 @@ k_tile_gather(const int32_t* __restrict__ perm, const int32_t* __restrict__ nbr,
   while (m) {
     const int t = __ffs(m) - 1;
     m &= m - 1;
-    if (threadIdx.x == 0) tile_taps[tile * 32 + s] = uint8_t(t);
     gidx[(off + s) * kTileRows + threadIdx.x] = v >= 0 ? nbr[int64_t(v) * kTaps + t] : -1;
     ++s;
   }
@@ -297,21 +283,82 @@ __global__ void k_group_keys(const uint32_t* __restrict__ tile_mask, int64_t n_t
   vals[i] = int32_t(g);
 }
 
-template <class T>
-int dev_alloc(T** p, size_t count, cudaStream_t s) {
-  *p = nullptr;
-  if (count == 0) count = 1;
-  if (cudaMallocAsync(reinterpret_cast<void**>(p), count * sizeof(T), s) != cudaSuccess) {
-    cudaGetLastError();
-    return SMC_ERR_OOM;
+// Tap-major tile lists (see Plan::tap_tiles), one block per tap.
+__global__ void __launch_bounds__(1024)
+k_tap_count(const uint32_t* __restrict__ tile_mask, int64_t n_tiles, int32_t* __restrict__ count) {
+  __shared__ int32_t part[32];
+  const int k = blockIdx.x;
+  int32_t c = 0;
+  for (int64_t t = threadIdx.x; t < n_tiles; t += blockDim.x) c += (tile_mask[t] >> k) & 1u;
+  c = __reduce_add_sync(0xffffffffu, c);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = c;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    int32_t v = threadIdx.x < blockDim.x / 32 ? part[threadIdx.x] : 0;
+    v = __reduce_add_sync(0xffffffffu, v);
+    if (threadIdx.x == 0) count[k] = v;
   }
-  return SMC_OK;
 }
 
-template <class T>
-void dev_free(T*& p, cudaStream_t s) {
-  if (p) cudaFreeAsync(p, s);
-  p = nullptr;
+__global__ void k_tap_scan(const int32_t* __restrict__ count, int32_t* __restrict__ tap_start,
+                           int32_t* __restrict__ tap_chunk, int chunk) {
+  if (threadIdx.x != 0) return;
+  int32_t s = 0, c = 0;
+  for (int k = 0; k < kTaps; ++k) {
+    tap_start[k] = s;
+    tap_chunk[k] = c;
+    s += count[k];
+    c += (count[k] + chunk - 1) / chunk;
+  }
+  tap_start[kTaps] = s;
+  tap_chunk[kTaps] = c;
+}
+
+__global__ void __launch_bounds__(1024)
+k_tap_fill(const uint32_t* __restrict__ tile_mask, const int32_t* __restrict__ tile_off,
+           int64_t n_tiles, const int32_t* __restrict__ tap_start, int2* __restrict__ tap_tiles) {
+  __shared__ int32_t wsum[32];
+  __shared__ int32_t base;
+  const int k = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) base = tap_start[k];
+  __syncthreads();
+  for (int64_t t0 = 0; t0 < n_tiles; t0 += blockDim.x) {
+    const int64_t t = t0 + threadIdx.x;
+    const uint32_t m = t < n_tiles ? tile_mask[t] : 0u;
+    const int has = (m >> k) & 1u;
+    const uint32_t ballot = __ballot_sync(0xffffffffu, has);
+    if (lane == 0) wsum[warp] = __popc(ballot);
+    __syncthreads();
+    int32_t before = 0, total = 0;
+    for (int w = 0; w < int(blockDim.x / 32); ++w) {
+      before += w < warp ? wsum[w] : 0;
+      total += wsum[w];
+    }
+    if (has) {
+      const int32_t pos = base + before + __popc(ballot & ((1u << lane) - 1u));
+      tap_tiles[pos] = make_int2(int(t), tile_off[t] + __popc(m & ((1u << k) - 1u)));
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) base += total;
+    __syncthreads();
+  }
+}
+
+// Work-item records in the sorted group order (see Plan::items).
+__global__ void k_item_records(const int32_t* __restrict__ order, int64_t n_groups, int G,
+                               const uint32_t* __restrict__ tile_mask,
+                               const int32_t* __restrict__ tile_off, int64_t n_tiles,
+                               int4* __restrict__ items) {
+  const int64_t q = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+  if (q >= n_groups) return;
+  const int64_t t = int64_t(order[q]) * G;
+  int4 r;
+  r.x = int(t);
+  r.y = int(tile_mask[t]);
+  r.z = (G == 2 && t + 1 < n_tiles) ? int(tile_mask[t + 1]) : 0;
+  r.w = tile_off[t];
+  items[q] = r;
 }
 
 inline unsigned grid_for(int64_t n, int threads) {
@@ -326,33 +373,71 @@ int status_from_device(int32_t dev) {
   return SMC_OK;
 }
 
+// Carves one allocation into 256-byte-aligned arrays.  A first pass with a
+// null base only measures.
+struct Carve {
+  uint8_t* base = nullptr;
+  size_t off = 0;
+  template <class T>
+  T* take(size_t count) {
+    off = (off + 255) & ~size_t(255);
+    T* p = reinterpret_cast<T*>(base + off);
+    off += (count ? count : 1) * sizeof(T);
+    return p;
+  }
+};
+
+// Device counters written by the build and read back once at its end.
+struct BuildCounters {
+  int32_t status;
+  uint32_t work_counter[63];   // the tensor-core kernel's item counter (+ finished CTAs)
+  unsigned long long stats[2];  // useful pairs, issued rows x taps
+};
+
+// The plan's arrays in one arena (sizes are upper bounds where they depend on
+// the tile masks, so nothing has to be read back before the end).
+void carve_plan(Carve& c, Plan* p, BuildCounters** ctr) {
+  const int64_t n = p->n, nt = p->n_tiles;
+  *ctr = c.take<BuildCounters>(1);
+  p->nbr = c.take<int32_t>(size_t(n) * kTaps);
+  p->mask = c.take<uint32_t>(size_t(n));
+  p->perm = c.take<int32_t>(size_t(n));
+  p->tile_mask = c.take<uint32_t>(size_t(nt));
+  p->tile_off = c.take<int32_t>(size_t(nt) + 1);
+  p->gidx = c.take<int32_t>(size_t(nt) * kTaps * kTileRows);
+  p->out_row = c.take<int32_t>(size_t(nt) * kTileRows);
+  p->items[0] = c.take<int4>(size_t(nt));
+  p->items[1] = c.take<int4>(size_t((nt + 1) / 2));
+  p->tap_tiles = c.take<int2>(size_t(nt) * kTaps);
+  p->tap_start = c.take<int32_t>(kTaps + 1);
+  p->tap_chunk = c.take<int32_t>(kTaps + 1);
+}
+
 struct Scratch {
-  uint64_t* keys = nullptr;
-  int32_t* vals = nullptr;
+  Slot* table = nullptr;
+  unsigned long long* ckeys[2] = {nullptr, nullptr};  // packed coordinates (sort lookup)
   uint32_t* skeys[2] = {nullptr, nullptr};
   int32_t* svals[2] = {nullptr, nullptr};
   uint32_t* hist = nullptr;
-  uint32_t* tile_ntaps = nullptr;
-  unsigned long long* stats = nullptr;
+  int32_t* tap_count = nullptr;
   uint32_t* gkeys[2] = {nullptr, nullptr};
   int32_t* gvals = nullptr;
-  uint32_t* ghist = nullptr;
-  void release(cudaStream_t s) {
-    dev_free(gkeys[0], s);
-    dev_free(gkeys[1], s);
-    dev_free(gvals, s);
-    dev_free(ghist, s);
-    dev_free(keys, s);
-    dev_free(vals, s);
-    for (int i = 0; i < 2; ++i) {
-      dev_free(skeys[i], s);
-      dev_free(svals[i], s);
-    }
-    dev_free(hist, s);
-    dev_free(tile_ntaps, s);
-    dev_free(stats, s);
-  }
+  int32_t* gorder = nullptr;
 };
+
+void carve_scratch(Carve& c, Scratch* sc, int64_t n, int64_t nt, uint64_t cap, bool sorted) {
+  sc->table = c.take<Slot>(sorted ? 0 : size_t(cap));
+  for (int i = 0; i < 2; ++i) sc->ckeys[i] = c.take<unsigned long long>(sorted ? size_t(n) : 0);
+  for (int i = 0; i < 2; ++i) {
+    sc->skeys[i] = c.take<uint32_t>(size_t(n));
+    sc->svals[i] = c.take<int32_t>(size_t(n));
+    sc->gkeys[i] = c.take<uint32_t>(size_t(nt));
+  }
+  sc->hist = c.take<uint32_t>(sort_hist_words(n));
+  sc->tap_count = c.take<int32_t>(kTaps);
+  sc->gvals = c.take<int32_t>(size_t(nt));
+  sc->gorder = c.take<int32_t>(size_t(nt));
+}
 
 #define SMC_TRY(expr)             \
   do {                            \
@@ -365,19 +450,7 @@ struct Scratch {
     if (cudaGetLastError() != cudaSuccess) return SMC_ERR_CUDA; \
   } while (0)
 
-int build_plan_impl(const int32_t* coords, int64_t n, int32_t stride, int64_t table_capacity,
-                    int32_t order, cudaStream_t s, Plan* plan, Scratch& sc) {
-  const int4* c4 = reinterpret_cast<const int4*>(coords);
-  SMC_TRY(dev_alloc(&plan->status, 1, s));
-  SMC_TRY(dev_alloc(&plan->work_counter, 64, s));
-  if (cudaMemsetAsync(plan->work_counter, 0, 64 * sizeof(uint32_t), s) != cudaSuccess)
-    return SMC_ERR_CUDA;
-  if (cudaMemsetAsync(plan->status, 0, sizeof(int32_t), s) != cudaSuccess) return SMC_ERR_CUDA;
-  plan->n = n;
-  plan->n_tiles = (n + kTileRows - 1) / kTileRows;
-  if (n == 0) return SMC_OK;
-
-  // 1. hash insert
+uint64_t table_slots(int64_t n, int64_t table_capacity) {
   uint64_t cap = 64;
   if (table_capacity > 0) {
     cap = 1;
@@ -387,42 +460,70 @@ int build_plan_impl(const int32_t* coords, int64_t n, int32_t stride, int64_t ta
   } else {
     while (cap < uint64_t(2 * n)) cap <<= 1;
   }
-  SMC_TRY(dev_alloc(&sc.keys, cap, s));
-  SMC_TRY(dev_alloc(&sc.vals, cap, s));
-  if (cudaMemsetAsync(sc.keys, 0xFF, cap * sizeof(uint64_t), s) != cudaSuccess) return SMC_ERR_CUDA;
-  k_insert<<<grid_for(n, 256), 256, 0, s>>>(c4, n, sc.keys, sc.vals, cap - 1, plan->status);
-  SMC_LAUNCHED();
+  return cap;
+}
 
-  // 2. neighbour map and masks
-  SMC_TRY(dev_alloc(&plan->nbr, size_t(n) * kTaps, s));
-  SMC_TRY(dev_alloc(&plan->mask, size_t(n), s));
-  k_neighbors<<<grid_for(n, kNbrVoxels), kNbrThreads, 0, s>>>(c4, n, stride, sc.keys, sc.vals,
-                                                               cap - 1, plan->nbr, plan->mask);
+int build_plan_impl(const int32_t* coords, int64_t n, int32_t stride, int64_t table_capacity,
+                    int32_t order, int32_t lookup, cudaStream_t s, Plan* plan,
+                    void** scratch_mem) {
+  const bool sorted = lookup == SMC_LOOKUP_SORT;
+  const int4* c4 = reinterpret_cast<const int4*>(coords);
+  plan->n = n;
+  plan->n_tiles = (n + kTileRows - 1) / kTileRows;
+  const int64_t nt = plan->n_tiles;
+  const uint64_t cap = n > 0 ? table_slots(n, table_capacity) : 1;
+
+  // two allocations: the plan's arena (kept) and the build's scratch (freed)
+  Carve pc;
+  BuildCounters* ctr = nullptr;
+  carve_plan(pc, plan, &ctr);
+  if (cudaMallocAsync(&plan->arena, pc.off, s) != cudaSuccess) {
+    cudaGetLastError();
+    plan->arena = nullptr;
+    return SMC_ERR_OOM;
+  }
+  pc = Carve{static_cast<uint8_t*>(plan->arena), 0};
+  carve_plan(pc, plan, &ctr);
+  plan->status = &ctr->status;
+  plan->work_counter = ctr->work_counter;
+  if (cudaMemsetAsync(ctr, 0, sizeof(BuildCounters), s) != cudaSuccess) return SMC_ERR_CUDA;
+  if (n == 0) return SMC_OK;
+
+  Carve scc;
+  Scratch sc;
+  carve_scratch(scc, &sc, n, nt, cap, sorted);
+  if (cudaMallocAsync(scratch_mem, scc.off, s) != cudaSuccess) {
+    cudaGetLastError();
+    *scratch_mem = nullptr;
+    return SMC_ERR_OOM;
+  }
+  scc = Carve{static_cast<uint8_t*>(*scratch_mem), 0};
+  carve_scratch(scc, &sc, n, nt, cap, sorted);
+
+  // 1. lookup structure; 2. neighbour map and masks
+  if (sorted) {
+    k_pack_keys<<<grid_for(n, 256), 256, 0, s>>>(c4, n, sc.ckeys[0], sc.svals[0], plan->status);
+    SMC_LAUNCHED();
+    int cur = 0;
+    SMC_TRY(radix_sort(sc.ckeys, sc.svals, 0, n, 64, sc.hist, s, &cur));
+    k_sorted_dups<<<grid_for(n, 256), 256, 0, s>>>(sc.ckeys[cur], n, plan->status);
+    k_neighbors_sorted<<<grid_for(n, kNbrVoxels), kNbrThreads, 0, s>>>(
+        c4, n, stride, sc.ckeys[cur], sc.svals[cur], plan->nbr, plan->mask);
+  } else {
+    if (cudaMemsetAsync(sc.table, 0xFF, cap * sizeof(Slot), s) != cudaSuccess)
+      return SMC_ERR_CUDA;
+    k_insert<<<grid_for(n, 256), 256, 0, s>>>(c4, n, sc.table, cap - 1, plan->status);
+    k_neighbors<<<grid_for(n, kNbrVoxels), kNbrThreads, 0, s>>>(c4, n, stride, sc.table, cap - 1,
+                                                                 plan->nbr, plan->mask);
+  }
   SMC_LAUNCHED();
-  dev_free(sc.keys, s);
-  dev_free(sc.vals, s);
 
   // 3. row order
-  SMC_TRY(dev_alloc(&plan->perm, size_t(n), s));
   if (order == SMC_ORDER_MASK) {
-    const int nblocks = int((n + kSortTile - 1) / kSortTile);
-    for (int i = 0; i < 2; ++i) {
-      SMC_TRY(dev_alloc(&sc.skeys[i], size_t(n), s));
-      SMC_TRY(dev_alloc(&sc.svals[i], size_t(n), s));
-    }
-    SMC_TRY(dev_alloc(&sc.hist, size_t(256) * nblocks, s));
     k_sort_keys<<<grid_for(n, 256), 256, 0, s>>>(plan->mask, n, sc.skeys[0], sc.svals[0]);
     SMC_LAUNCHED();
     int cur = 0;
-    for (int shift = 0; shift < 32; shift += 8) {
-      k_radix_hist<<<nblocks, kSortThreads, 0, s>>>(sc.skeys[cur], n, shift, sc.hist, nblocks);
-      k_scan_exclusive<<<1, 1024, 0, s>>>(sc.hist, int64_t(256) * nblocks);
-      k_radix_scatter<<<nblocks, kSortThreads, 0, s>>>(sc.skeys[cur], sc.svals[cur],
-                                                       sc.skeys[cur ^ 1], sc.svals[cur ^ 1], n,
-                                                       shift, sc.hist, nblocks);
-      SMC_LAUNCHED();
-      cur ^= 1;
-    }
+    SMC_TRY(radix_sort(sc.skeys, sc.svals, 0, n, 32, sc.hist, s, &cur));
     if (cudaMemcpyAsync(plan->perm, sc.svals[cur], size_t(n) * sizeof(int32_t),
                         cudaMemcpyDeviceToDevice, s) != cudaSuccess)
       return SMC_ERR_CUDA;
@@ -431,29 +532,49 @@ int build_plan_impl(const int32_t* coords, int64_t n, int32_t stride, int64_t ta
     SMC_LAUNCHED();
   }
 
-  // 4. tile plan
-  const int64_t nt = plan->n_tiles;
-  SMC_TRY(dev_alloc(&plan->tile_mask, size_t(nt), s));
-  SMC_TRY(dev_alloc(&sc.tile_ntaps, size_t(nt) + 1, s));
-  SMC_TRY(dev_alloc(&sc.stats, 2, s));
-  if (cudaMemsetAsync(sc.tile_ntaps, 0, (size_t(nt) + 1) * sizeof(uint32_t), s) != cudaSuccess ||
-      cudaMemsetAsync(sc.stats, 0, 2 * sizeof(unsigned long long), s) != cudaSuccess)
-    return SMC_ERR_CUDA;
+  // 4. tile plan: masks and tap counts, slot offsets, gather index
   k_tile_mask<<<unsigned(nt), kTileRows, 0, s>>>(plan->perm, plan->mask, n, plan->tile_mask,
-                                                  sc.tile_ntaps, sc.stats);
-  k_scan_exclusive<<<1, 1024, 0, s>>>(sc.tile_ntaps, nt + 1);
+                                                  reinterpret_cast<uint32_t*>(plan->tile_off),
+                                                  ctr->stats);
+  if (cudaMemsetAsync(plan->tile_off + nt, 0, sizeof(int32_t), s) != cudaSuccess)
+    return SMC_ERR_CUDA;
+  SMC_TRY(scan_exclusive(reinterpret_cast<uint32_t*>(plan->tile_off), nt + 1, s));
+  k_tile_gather<<<unsigned(nt), kTileRows, 0, s>>>(plan->perm, plan->nbr, n, plan->tile_mask,
+                                                    plan->tile_off, plan->gidx, plan->out_row);
   SMC_LAUNCHED();
 
+  // tap-major tile lists for the weight gradient
+  k_tap_count<<<kTaps, 1024, 0, s>>>(plan->tile_mask, nt, sc.tap_count);
+  k_tap_scan<<<1, 32, 0, s>>>(sc.tap_count, plan->tap_start, plan->tap_chunk, kBwdChunk);
+  k_tap_fill<<<kTaps, 1024, 0, s>>>(plan->tile_mask, plan->tile_off, nt, plan->tap_start,
+                                    plan->tap_tiles);
+  SMC_LAUNCHED();
+
+  // 5. work items of one and two tiles, most taps first: one stable radix
+  // pass over the (27 - tap count) keys, which are below 256
+  for (int G = 1; G <= 2; ++G) {
+    const int64_t ng = (nt + G - 1) / G;
+    k_group_keys<<<grid_for(ng, 256), 256, 0, s>>>(plan->tile_mask, nt, G, ng, sc.gkeys[0],
+                                                    sc.gvals);
+    int32_t* gv[2] = {sc.gvals, sc.gorder};
+    int gcur = 0;
+    SMC_TRY(radix_sort(sc.gkeys, gv, 0, ng, 8, sc.hist, s, &gcur));
+    k_item_records<<<grid_for(ng, 256), 256, 0, s>>>(gv[gcur], ng, G, plan->tile_mask,
+                                                      plan->tile_off, nt, plan->items[G - 1]);
+    SMC_LAUNCHED();
+  }
+
+  // the one read-back: status word, plan counters, slot count
   struct {
-    uint32_t total;
     int32_t status;
+    int32_t total;
     unsigned long long stats[2];
   } h{};
-  if (cudaMemcpyAsync(&h.total, sc.tile_ntaps + nt, sizeof(uint32_t), cudaMemcpyDeviceToHost, s) !=
+  if (cudaMemcpyAsync(&h.status, plan->status, sizeof(int32_t), cudaMemcpyDeviceToHost, s) !=
           cudaSuccess ||
-      cudaMemcpyAsync(&h.status, plan->status, sizeof(int32_t), cudaMemcpyDeviceToHost, s) !=
+      cudaMemcpyAsync(&h.total, plan->tile_off + nt, sizeof(int32_t), cudaMemcpyDeviceToHost, s) !=
           cudaSuccess ||
-      cudaMemcpyAsync(h.stats, sc.stats, sizeof(h.stats), cudaMemcpyDeviceToHost, s) !=
+      cudaMemcpyAsync(h.stats, ctr->stats, sizeof(h.stats), cudaMemcpyDeviceToHost, s) !=
           cudaSuccess ||
       cudaStreamSynchronize(s) != cudaSuccess)
     return SMC_ERR_CUDA;
@@ -461,72 +582,35 @@ int build_plan_impl(const int32_t* coords, int64_t n, int32_t stride, int64_t ta
   plan->total_slots = h.total;
   plan->useful_pairs = int64_t(h.stats[0]);
   plan->issued_rows_taps = int64_t(h.stats[1]);
-  plan->tile_off = reinterpret_cast<int32_t*>(sc.tile_ntaps);  // ownership moves to the plan
-  sc.tile_ntaps = nullptr;
-
-  SMC_TRY(dev_alloc(&plan->tile_taps, size_t(nt) * 32, s));
-  SMC_TRY(dev_alloc(&plan->gidx, size_t(plan->total_slots) * kTileRows, s));
-  SMC_TRY(dev_alloc(&plan->out_row, size_t(nt) * kTileRows, s));
-  k_tile_gather<<<unsigned(nt), kTileRows, 0, s>>>(plan->perm, plan->nbr, n, plan->tile_mask,
-                                                    plan->tile_off, plan->tile_taps, plan->gidx,
-                                                    plan->out_row);
-  SMC_LAUNCHED();
-
-  // 5. work-item order for one and two tiles per item: one stable radix pass
-  // over the (27 - tap count) keys, which are below 256
-  {
-    const int gblocks = int((nt + kSortTile - 1) / kSortTile);
-    SMC_TRY(dev_alloc(&sc.gkeys[0], size_t(nt), s));
-    SMC_TRY(dev_alloc(&sc.gkeys[1], size_t(nt), s));
-    SMC_TRY(dev_alloc(&sc.gvals, size_t(nt), s));
-    SMC_TRY(dev_alloc(&sc.ghist, size_t(256) * gblocks, s));
-    for (int G = 1; G <= 2; ++G) {
-      const int64_t ng = (nt + G - 1) / G;
-      const int nb = int((ng + kSortTile - 1) / kSortTile);
-      SMC_TRY(dev_alloc(&plan->group_order[G - 1], size_t(ng), s));
-      k_group_keys<<<grid_for(ng, 256), 256, 0, s>>>(plan->tile_mask, nt, G, ng, sc.gkeys[0],
-                                                      sc.gvals);
-      k_radix_hist<<<nb, kSortThreads, 0, s>>>(sc.gkeys[0], ng, 0, sc.ghist, nb);
-      k_scan_exclusive<<<1, 1024, 0, s>>>(sc.ghist, int64_t(256) * nb);
-      k_radix_scatter<<<nb, kSortThreads, 0, s>>>(sc.gkeys[0], sc.gvals, sc.gkeys[1],
-                                                  plan->group_order[G - 1], ng, 0, sc.ghist, nb);
-      SMC_LAUNCHED();
-    }
-  }
-  if (cudaStreamSynchronize(s) != cudaSuccess) return SMC_ERR_CUDA;
   return SMC_OK;
 }
 
 }  // namespace
 
 void free_plan(Plan* plan) {
-  cudaStream_t s = nullptr;
-  dev_free(plan->nbr, s);
-  dev_free(plan->mask, s);
-  dev_free(plan->perm, s);
-  dev_free(plan->tile_mask, s);
-  dev_free(plan->tile_off, s);
-  dev_free(plan->tile_taps, s);
-  dev_free(plan->gidx, s);
-  dev_free(plan->out_row, s);
-  dev_free(plan->status, s);
-  dev_free(plan->work_counter, s);
-  dev_free(plan->group_order[0], s);
-  dev_free(plan->group_order[1], s);
-  cudaStreamSynchronize(s);
+  // A forward queued on any stream (including non-blocking ones, which the
+  // legacy stream does not order) may still read the plan: wait for all work
+  // on the device before handing the buffers back.
+  cudaDeviceSynchronize();
+  cudaGetLastError();
+  if (plan->arena) {
+    cudaFreeAsync(plan->arena, nullptr);
+    cudaStreamSynchronize(nullptr);
+  }
+  *plan = Plan{};
 }
 
 int build_plan(const int32_t* coords, int64_t n, int32_t stride, int64_t table_capacity,
-               int32_t order, cudaStream_t stream, Plan* plan) {
-  Scratch sc;
-  int rc = build_plan_impl(coords, n, stride, table_capacity, order, stream, plan, sc);
-  sc.release(stream);
+               int32_t order, int32_t lookup, cudaStream_t stream, Plan* plan) {
+  void* scratch = nullptr;
+  int rc = build_plan_impl(coords, n, stride, table_capacity, order, lookup, stream, plan,
+                           &scratch);
+  if (scratch) cudaFreeAsync(scratch, stream);  // stream-ordered after the build's kernels
   if (rc != SMC_OK) {
     cudaGetLastError();
+    cudaStreamSynchronize(stream);
     free_plan(plan);
-    *plan = Plan{};
   }
-  cudaStreamSynchronize(stream);
   return rc;
 }
 
@@ -540,6 +624,8 @@ int build_plan(const int32_t* coords, int64_t n, int32_t stride, int64_t table_c
 // table in a fixed-size array of static device memory that every device
 // loading this library reserves once, for the life of the process.
 // ---------------------------------------------------------------------------
+#include <cuda.h>
+
 #include <mutex>
 
 namespace smc {
@@ -549,8 +635,7 @@ constexpr int64_t kStaticMaxVoxels = SMC_STATIC_MAX_VOXELS;
 constexpr int64_t kStaticSlots = 2 * kStaticMaxVoxels;  // load factor <= 1/2
 
 struct StaticScratch {
-  uint64_t keys[kStaticSlots];
-  int32_t vals[kStaticSlots];
+  Slot table[kStaticSlots];
   uint32_t mask[kStaticMaxVoxels];
   int32_t status;
 };
@@ -562,7 +647,39 @@ static __device__ __align__(256) StaticScratch g_static_scratch;
 constexpr int kMaxDevices = 128;
 std::mutex g_static_mutex;
 StaticScratch* g_static_ptr[kMaxDevices] = {};
+unsigned long long g_static_ctx[kMaxDevices] = {};  // context the address belongs to
 
+// Unique id of the calling thread's current CUDA context (0 when the driver
+// cannot tell).  A device address is only valid in the context it came from;
+// after cudaDeviceReset the device gets a new context with a new id.
+unsigned long long current_context_id() {
+  using GetCurrent = CUresult (*)(CUcontext*);
+  using GetId = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCurrent get_current = nullptr;
+  static GetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrent>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetId>(p);
+    cudaGetLastError();
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of the static scratch array on the current device.  The
+// lookup runs once per device and context (with that device current); when
+// the context id is unknown it runs on every call.
 int static_scratch(StaticScratch** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) {
@@ -570,14 +687,19 @@ int static_scratch(StaticScratch** out) {
     return SMC_ERR_CUDA;
   }
   if (dev < 0 || dev >= kMaxDevices) return SMC_ERR_UNSUPPORTED;
+  // 0 before the thread's first CUDA call that binds a context: then the
+  // lookup below (which binds it) runs and records the id it ran under
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lock(g_static_mutex);
-  if (!g_static_ptr[dev]) {
+  if (!g_static_ptr[dev] || ctx == 0 || g_static_ctx[dev] != ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) {
       cudaGetLastError();
+      g_static_ptr[dev] = nullptr;
       return SMC_ERR_CUDA;
     }
     g_static_ptr[dev] = static_cast<StaticScratch*>(p);
+    g_static_ctx[dev] = current_context_id();
   }
   *out = g_static_ptr[dev];
   return SMC_OK;
@@ -602,13 +724,13 @@ extern "C" int smc_build_neighbor_map_static(const int32_t* coords_dev, int64_t 
   while (cap < uint64_t(2 * n)) cap <<= 1;
   // The array keeps the previous call's contents: reset the slots this call
   // probes and the status word before use.
-  if (cudaMemsetAsync(sc->keys, 0xFF, cap * sizeof(uint64_t), s) != cudaSuccess ||
+  if (cudaMemsetAsync(sc->table, 0xFF, cap * sizeof(Slot), s) != cudaSuccess ||
       cudaMemsetAsync(&sc->status, 0, sizeof(int32_t), s) != cudaSuccess)
     return SMC_ERR_CUDA;
   const int4* c4 = reinterpret_cast<const int4*>(coords_dev);
-  k_insert<<<grid_for(n, 256), 256, 0, s>>>(c4, n, sc->keys, sc->vals, cap - 1, &sc->status);
-  k_neighbors<<<grid_for(n, kNbrVoxels), kNbrThreads, 0, s>>>(c4, n, stride, sc->keys, sc->vals,
-                                                               cap - 1, map_dev, sc->mask);
+  k_insert<<<grid_for(n, 256), 256, 0, s>>>(c4, n, sc->table, cap - 1, &sc->status);
+  k_neighbors<<<grid_for(n, kNbrVoxels), kNbrThreads, 0, s>>>(c4, n, stride, sc->table, cap - 1,
+                                                               map_dev, sc->mask);
   if (cudaGetLastError() != cudaSuccess) return SMC_ERR_CUDA;
   int32_t dev_status = 0;
   if (cudaMemcpyAsync(&dev_status, &sc->status, sizeof(int32_t), cudaMemcpyDeviceToHost, s) !=

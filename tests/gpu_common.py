@@ -29,24 +29,40 @@ def as_f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().to("cpu", torch.float64).numpy()
 
 
-def check_conv(out_gpu: torch.Tensor, ref: np.ndarray, scale: np.ndarray, what: str = "") -> dict:
-    out = as_f64(out_gpu)
-    assert out.shape == ref.shape, (out.shape, ref.shape)
-    assert np.all(np.isfinite(out)), f"{what}: non-finite output"
-    err = np.abs(out - ref)
-    if out_gpu.dtype == torch.float32:
-        bound = F32_RTOL * np.abs(ref) + F32_FLOOR * scale
-    else:
-        bound = HALF_TOL * scale + UNIT_ROUNDOFF[out_gpu.dtype] * np.abs(ref)
-    bad = err > bound
-    if bad.any():
-        idx = np.argwhere(bad)[:5]
-        detail = [(tuple(int(v) for v in i), float(out[tuple(i)]), float(ref[tuple(i)]),
-                   float(scale[tuple(i)])) for i in idx]
-        raise AssertionError(f"{what}: {int(bad.sum())} elements out of tolerance, e.g. {detail}")
-    with np.errstate(divide="ignore", invalid="ignore"):
-        ratio = np.where(scale > 0, err / scale, 0.0)
-    return {"max_err_over_scale": float(ratio.max()) if ratio.size else 0.0}
+def check_conv(out_gpu: torch.Tensor, ref: np.ndarray, scale: np.ndarray, what: str = "",
+               chunk: int = 1 << 18, input_dtype=None) -> dict:
+    """Element-wise tolerance check of a GPU result against the oracle, in row
+    chunks (full-size workloads hold millions of rows).  input_dtype, when the
+    result is fp32 but its inputs were half precision (the weight gradient),
+    selects the half-precision bound without an output-rounding term."""
+    assert tuple(out_gpu.shape) == ref.shape, (tuple(out_gpu.shape), ref.shape)
+    worst = 0.0
+    n_bad = 0
+    detail = []
+    for r0 in range(0, ref.shape[0], chunk):
+        out = as_f64(out_gpu[r0:r0 + chunk])
+        rf, sc = ref[r0:r0 + chunk], scale[r0:r0 + chunk]
+        assert np.all(np.isfinite(out)), f"{what}: non-finite output"
+        err = np.abs(out - rf)
+        if input_dtype in (torch.float16, torch.bfloat16):
+            bound = HALF_TOL * sc  # fp32 result: its own rounding is far below the bound
+        elif out_gpu.dtype == torch.float32:
+            bound = F32_RTOL * np.abs(rf) + F32_FLOOR * sc
+        else:
+            bound = HALF_TOL * sc + UNIT_ROUNDOFF[out_gpu.dtype] * np.abs(rf)
+        bad = err > bound
+        if bad.any():
+            n_bad += int(bad.sum())
+            for i in np.argwhere(bad)[:5 - len(detail)]:
+                detail.append(((r0 + int(i[0]), int(i[1])), float(out[tuple(i)]),
+                               float(rf[tuple(i)]), float(sc[tuple(i)])))
+        with np.errstate(divide="ignore", invalid="ignore"):
+            ratio = np.where(sc > 0, err / sc, 0.0)
+        if ratio.size:
+            worst = max(worst, float(ratio.max()))
+    if n_bad:
+        raise AssertionError(f"{what}: {n_bad} elements out of tolerance, e.g. {detail}")
+    return {"max_err_over_scale": worst}
 
 
 def oracle_conv(coords: np.ndarray, feats: torch.Tensor, W: torch.Tensor, K: int, rows=None,
@@ -54,13 +70,3 @@ def oracle_conv(coords: np.ndarray, feats: torch.Tensor, W: torch.Tensor, K: int
     if nbr is None:
         nbr = native.neighbor_map(coords, K, stride)
     return native.submconv(as_f64(feats), as_f64(W), nbr, rows=rows)
-
-
-def sample_rows(n: int, count: int, seed: int = 0) -> np.ndarray:
-    """Sorted sample of row ids that always includes the first and last rows."""
-    if count >= n:
-        return np.arange(n, dtype=np.int64)
-    rng = np.random.default_rng(seed)
-    rows = rng.choice(n, size=count, replace=False)
-    rows = np.unique(np.concatenate([rows, [0, n - 1]]))
-    return rows.astype(np.int64)
