@@ -266,6 +266,36 @@ int smc_downsample2(const int32_t* coords_dev, int64_t n, const void* feats_dev,
 int smc_subdivide2(const int32_t* coords_dev, int64_t n, const void* feats_dev, int c, int dtype,
                    int32_t* out_coords_dev, void* out_feats_dev, smc_stream_t stream);
 
+/* Activation of the fused epilogue (smc_epilogue.activation). */
+enum smc_activation {
+  SMC_ACT_NONE = 0,
+  SMC_ACT_RELU = 1, /* max(v, 0) */
+  SMC_ACT_SILU = 2, /* v / (1 + exp(-v)) */
+  SMC_ACT_GELU = 3  /* v / 2 * (1 + erf(v / sqrt 2)), the exact form */
+};
+
+/* Element-wise work fused into the convolution's epilogue. */
+typedef struct smc_epilogue {
+  const void* bias;     /* device pointer, [cout] of dtype, or NULL */
+  const void* residual; /* device pointer, [n][cout] of dtype, or NULL; may not
+                           overlap out */
+  int32_t activation;   /* enum smc_activation */
+  int32_t reserved;     /* must be 0 */
+} smc_epilogue;
+
+/*
+ * smc_forward with a fused epilogue: out = act(conv + bias) + residual,
+ * computed on the fp32 (fp64 for SMC_F32) accumulator before the one rounding
+ * to dtype.  This is the layer shape of the sparse ResBlock (trellis_sparse_mlx
+ * README, "What's in it": SparseLinear, SparseSiLU/GELU, SparseResBlock): a
+ * convolution with bias, followed by an activation or closed by the skip
+ * connection's sum, in one pass over the output.  ep == NULL is smc_forward.
+ * Errors: as smc_forward; SMC_ERR_INVALID also for a bad activation, a
+ * non-zero reserved field or misaligned bias / residual pointers.
+ */
+int smc_forward_ex(smc_handle_t h, const void* feats, const void* W, void* out, int K, int cin,
+                   int cout, int dtype, const smc_epilogue* ep, smc_stream_t stream);
+
 /* Copy the int32 [n][27] neighbour map (-1 = no active neighbour) into
  * map_dev, asynchronously on stream.  Entry [i][k] is the row j whose
  * coordinates are coords[i] + stride * d(k) in the same batch: the indice map

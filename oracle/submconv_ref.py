@@ -194,3 +194,38 @@ def subdivide2(coords, feats):
                     out_c[c] = (b, 2 * x + dx, 2 * y + dy, 2 * z + dz)
                     out_f[c] = f[i]
     return out_c, out_f
+
+
+# ----------------------------------------------------------------------------
+# Fused epilogue of a convolution layer inside a sparse ResBlock
+# (trellis_sparse_mlx README, "What's in it": SparseLinear, SparseSiLU/GELU,
+# SparseResBlock).  Reading: out = act(conv + bias) + residual, every term
+# optional; SiLU(v) = v / (1 + exp(-v)); GELU is the exact (erf) form,
+# v / 2 * (1 + erf(v / sqrt(2))); ReLU(v) = max(v, 0).
+# ----------------------------------------------------------------------------
+ACTIVATIONS = ("none", "relu", "silu", "gelu")
+
+
+def activation(v: np.ndarray, act: str) -> np.ndarray:
+    v = np.asarray(v, dtype=np.float64)
+    if act == "none":
+        return v
+    if act == "relu":
+        return np.maximum(v, 0.0)
+    if act == "silu":
+        return v / (1.0 + np.exp(-v))
+    if act == "gelu":
+        from math import erf, sqrt
+        return 0.5 * v * (1.0 + np.vectorize(erf)(v / sqrt(2.0)))
+    raise ValueError(act)
+
+
+def epilogue(conv_out, bias=None, act: str = "none", residual=None) -> np.ndarray:
+    """act(conv_out + bias) + residual in float64 (bias [Cout], residual [N, Cout])."""
+    v = np.asarray(conv_out, dtype=np.float64)
+    if bias is not None:
+        v = v + np.asarray(bias, dtype=np.float64)[None, :]
+    v = activation(v, act)
+    if residual is not None:
+        v = v + np.asarray(residual, dtype=np.float64)
+    return v

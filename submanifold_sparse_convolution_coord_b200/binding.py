@@ -33,6 +33,7 @@ EXPORTS = (
     "smc_get_plan_stats", "smc_get_sizes", "smc_get_tile_plan", "smc_device_status",
     "smc_destroy", "smc_status_string", "smc_version", "smc_build_neighbor_map_static",
     "smc_backward_input", "smc_backward_weight", "smc_downsample2", "smc_subdivide2",
+    "smc_forward_ex",
 )
 
 
@@ -40,6 +41,14 @@ class SmcError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
         super().__init__(f"{where}: {STATUS.get(status, status)} ({status_string(status)})")
+
+
+ACT_CODE = {"none": 0, "relu": 1, "silu": 2, "gelu": 3}
+
+
+class _Epilogue(ctypes.Structure):
+    _fields_ = [("bias", ctypes.c_void_p), ("residual", ctypes.c_void_p),
+                ("activation", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 class _Options(ctypes.Structure):
@@ -64,6 +73,7 @@ def lib() -> ctypes.CDLL:
     L.smc_build_index.argtypes = [p, i64, i32, ctypes.POINTER(p)]
     L.smc_build_index_ex.argtypes = [p, i64, i32, ctypes.POINTER(_Options), p, ctypes.POINTER(p)]
     L.smc_forward.argtypes = [p, p, p, p, i, i, i, i, p]
+    L.smc_forward_ex.argtypes = [p, p, p, p, i, i, i, i, ctypes.POINTER(_Epilogue), p]
     L.smc_backward_input.argtypes = [p, p, p, p, i, i, i, i, p]
     L.smc_backward_weight.argtypes = [p, p, p, p, i, i, i, i, p]
     L.smc_downsample2.argtypes = [p, i64, p, i, i, p, p, ctypes.POINTER(i64), p]
@@ -146,6 +156,27 @@ def smc_forward(handle: int, feats: torch.Tensor, W: torch.Tensor, out: torch.Te
                                ctypes.c_void_p(op), int(K), int(cin), int(cout),
                                DTYPE_CODE[dtype], _stream(stream, feats.device))
     _check(rc, "smc_forward")
+
+
+def smc_forward_ex(handle: int, feats: torch.Tensor, W: torch.Tensor, out: torch.Tensor, K: int,
+                   cin: int, cout: int, bias: Optional[torch.Tensor] = None,
+                   residual: Optional[torch.Tensor] = None, activation: str = "none",
+                   stream: Optional[torch.cuda.Stream] = None) -> None:
+    """smc_forward with the fused epilogue out = act(conv + bias) + residual."""
+    dtype = feats.dtype
+    if dtype not in DTYPE_CODE:
+        raise ValueError(f"unsupported dtype {dtype}")
+    fp = _dev_ptr(feats, "feats", dtype)
+    wp = _dev_ptr(W, "W", dtype)
+    op = _dev_ptr(out, "out", dtype)
+    bp = _dev_ptr(bias, "bias", dtype) if bias is not None else None
+    rp = _dev_ptr(residual, "residual", dtype) if residual is not None else None
+    ep = _Epilogue(bp, rp, ACT_CODE[activation], 0)
+    with torch.cuda.device(feats.device):
+        rc = lib().smc_forward_ex(ctypes.c_void_p(handle), ctypes.c_void_p(fp), ctypes.c_void_p(wp),
+                                  ctypes.c_void_p(op), int(K), int(cin), int(cout),
+                                  DTYPE_CODE[dtype], ctypes.byref(ep), _stream(stream, feats.device))
+    _check(rc, "smc_forward_ex")
 
 
 def smc_backward_input(handle: int, grad_out: torch.Tensor, W: torch.Tensor,
@@ -314,7 +345,9 @@ class SubMIndex:
         return smc_device_status(self.handle, self.device)
 
     def forward(self, feats: torch.Tensor, W: torch.Tensor, K: int = 3,
-                out: Optional[torch.Tensor] = None) -> torch.Tensor:
+                out: Optional[torch.Tensor] = None, bias: Optional[torch.Tensor] = None,
+                residual: Optional[torch.Tensor] = None, activation: str = "none") -> torch.Tensor:
+        """act(conv(feats, W) + bias) + residual (the epilogue parts are optional)."""
         if feats.dim() != 2 or feats.shape[0] != self.n:
             raise ValueError("feats must be [N, Cin] for this index")
         taps, cin, cout = W.shape
@@ -322,7 +355,10 @@ class SubMIndex:
             raise ValueError("W must be [K^3, Cin, Cout]")
         if out is None:
             out = torch.empty((self.n, cout), dtype=feats.dtype, device=feats.device)
-        smc_forward(self.handle, feats, W, out, K, cin, cout)
+        if bias is None and residual is None and activation == "none":
+            smc_forward(self.handle, feats, W, out, K, cin, cout)
+        else:
+            smc_forward_ex(self.handle, feats, W, out, K, cin, cout, bias, residual, activation)
         return out
 
 

@@ -62,10 +62,10 @@ int check_call(smc_index* h, int K, int cin, int cout, int dtype) {
 }
 
 int conv(const smc::Plan& plan, bool dense, const void* x, const void* W, void* y, int cin,
-         int cout, int dtype, cudaStream_t s) {
+         int cout, int dtype, const smc::Epilogue& ep, cudaStream_t s) {
   if (smc::conv_tc_supported(cin, cout, dtype))
-    return smc::launch_conv_tc(plan, dense, x, W, y, cin, cout, dtype, s);
-  return smc::launch_conv_simt(plan, dense, x, W, y, cin, cout, dtype, s);
+    return smc::launch_conv_tc(plan, dense, x, W, y, cin, cout, dtype, ep, s);
+  return smc::launch_conv_simt(plan, dense, x, W, y, cin, cout, dtype, ep, s);
 }
 
 }  // namespace
@@ -140,16 +140,31 @@ int smc_build_index(const int32_t* coords_dev, int64_t n, int32_t stride,
   return smc_build_index_ex(coords_dev, n, stride, nullptr, nullptr, out_handle);
 }
 
-int smc_forward(smc_handle_t h, const void* feats, const void* W, void* out, int K, int cin,
-                int cout, int dtype, smc_stream_t stream) {
+int smc_forward_ex(smc_handle_t h, const void* feats, const void* W, void* out, int K, int cin,
+                   int cout, int dtype, const smc_epilogue* ep, smc_stream_t stream) {
   const int rc = check_call(h, K, cin, cout, dtype);
   if (rc != SMC_OK) return rc;
+  smc::Epilogue e;
+  if (ep) {
+    if (ep->reserved != 0 || ep->activation < SMC_ACT_NONE || ep->activation > SMC_ACT_GELU)
+      return SMC_ERR_INVALID;
+    if ((ep->bias && !aligned16(ep->bias)) || (ep->residual && !aligned16(ep->residual)))
+      return SMC_ERR_INVALID;
+    e.bias = ep->bias;
+    e.residual = ep->residual;
+    e.act = ep->activation;
+  }
   const smc::Plan& plan = h->plan;
   if (plan.n == 0) return SMC_OK;
   if (!feats || !W || !out) return SMC_ERR_INVALID;
   if (!aligned16(feats) || !aligned16(W) || !aligned16(out)) return SMC_ERR_INVALID;
-  return conv(plan, K == 1, feats, W, out, cin, cout, dtype,
+  return conv(plan, K == 1, feats, W, out, cin, cout, dtype, e,
               reinterpret_cast<cudaStream_t>(stream));
+}
+
+int smc_forward(smc_handle_t h, const void* feats, const void* W, void* out, int K, int cin,
+                int cout, int dtype, smc_stream_t stream) {
+  return smc_forward_ex(h, feats, W, out, K, cin, cout, dtype, nullptr, stream);
 }
 
 int smc_backward_input(smc_handle_t h, const void* grad_out, const void* W, void* grad_in, int K,
@@ -167,7 +182,7 @@ int smc_backward_input(smc_handle_t h, const void* grad_out, const void* W, void
   // grad_in = conv(grad_out, W'), W'[k] = W[taps - 1 - k]^T: [taps][cout][cin]
   rc = smc::launch_weight_transpose(W, h->work, taps, cin, cout, dtype, s);
   if (rc != SMC_OK) return rc;
-  return conv(plan, K == 1, grad_out, h->work, grad_in, cout, cin, dtype, s);
+  return conv(plan, K == 1, grad_out, h->work, grad_in, cout, cin, dtype, smc::Epilogue{}, s);
 }
 
 int smc_backward_weight(smc_handle_t h, const void* feats, const void* grad_out, float* dW, int K,

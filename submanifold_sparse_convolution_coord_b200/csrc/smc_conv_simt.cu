@@ -7,7 +7,8 @@
 // each input voxel sums feats[c+d] @ W[d] over its active neighbours.)
 // Accumulation runs in tap order, then input-channel order: in fp64 for fp32
 // features (so the fp32 result is the exact sum rounded once), in fp32 FMA for
-// fp16/bf16 features.  One thread
+// fp16/bf16 features.  The optional epilogue act(acc + bias) + residual runs
+// in the accumulator's precision before the one rounding.  One thread
 // per (row, output channel); a block is 32 output channels x 8 rows, so the
 // weight reads of a warp are consecutive and the feature reads are broadcasts.
 #include <cuda_bf16.h>
@@ -56,10 +57,36 @@ struct Acc<float> {
   using type = double;
 };
 
+__device__ __forceinline__ float act_apply(float v, int act) {
+  switch (act) {
+    case SMC_ACT_RELU:
+      return fmaxf(v, 0.f);
+    case SMC_ACT_SILU:
+      return v / (1.f + expf(-v));
+    case SMC_ACT_GELU:
+      return 0.5f * v * (1.f + erff(v * 0.7071067811865476f));
+    default:
+      return v;
+  }
+}
+__device__ __forceinline__ double act_apply(double v, int act) {
+  switch (act) {
+    case SMC_ACT_RELU:
+      return fmax(v, 0.0);
+    case SMC_ACT_SILU:
+      return v / (1.0 + exp(-v));
+    case SMC_ACT_GELU:
+      return 0.5 * v * (1.0 + erf(v * 0.7071067811865476));
+    default:
+      return v;
+  }
+}
+
 template <class T>
 __global__ void __launch_bounds__(256)
 k_conv_simt(const T* __restrict__ feats, const T* __restrict__ W, T* __restrict__ out,
-            const int32_t* __restrict__ nbr, int64_t n, int cin, int cout, int dense) {
+            const int32_t* __restrict__ nbr, int64_t n, int cin, int cout, int dense,
+            const T* __restrict__ bias, const T* __restrict__ residual, int act) {
   const int64_t i = blockIdx.x * int64_t(blockDim.y) + threadIdx.y;
   const int co = blockIdx.y * blockDim.x + threadIdx.x;
   if (i >= n || co >= cout) return;
@@ -74,32 +101,36 @@ k_conv_simt(const T* __restrict__ feats, const T* __restrict__ W, T* __restrict_
     for (int ci = 0; ci < cin; ++ci)
       acc = fma(A(to_f(f[ci])), A(to_f(w[int64_t(ci) * cout])), acc);
   }
+  if (bias) acc += A(to_f(bias[co]));
+  acc = act_apply(acc, act);
+  if (residual) acc += A(to_f(residual[i * cout + co]));
   out[i * cout + co] = from_f<T>(float(acc));
 }
 
 template <class T>
 int launch_t(const Plan& plan, bool dense, const void* feats, const void* W, void* out, int cin,
-             int cout, cudaStream_t stream) {
+             int cout, const Epilogue& ep, cudaStream_t stream) {
   dim3 block(32, 8);
   dim3 grid(unsigned((plan.n + 7) / 8), unsigned((cout + 31) / 32));
-  k_conv_simt<T><<<grid, block, 0, stream>>>(static_cast<const T*>(feats),
-                                            static_cast<const T*>(W), static_cast<T*>(out),
-                                            plan.nbr, plan.n, cin, cout, dense ? 1 : 0);
+  k_conv_simt<T><<<grid, block, 0, stream>>>(
+      static_cast<const T*>(feats), static_cast<const T*>(W), static_cast<T*>(out), plan.nbr,
+      plan.n, cin, cout, dense ? 1 : 0, static_cast<const T*>(ep.bias),
+      static_cast<const T*>(ep.residual), ep.act);
   return cudaGetLastError() == cudaSuccess ? SMC_OK : SMC_ERR_CUDA;
 }
 
 }  // namespace
 
 int launch_conv_simt(const Plan& plan, bool dense, const void* feats, const void* W, void* out,
-                     int cin, int cout, int dtype, cudaStream_t stream) {
+                     int cin, int cout, int dtype, const Epilogue& ep, cudaStream_t stream) {
   if (plan.n == 0) return SMC_OK;
   switch (dtype) {
     case SMC_F32:
-      return launch_t<float>(plan, dense, feats, W, out, cin, cout, stream);
+      return launch_t<float>(plan, dense, feats, W, out, cin, cout, ep, stream);
     case SMC_F16:
-      return launch_t<__half>(plan, dense, feats, W, out, cin, cout, stream);
+      return launch_t<__half>(plan, dense, feats, W, out, cin, cout, ep, stream);
     case SMC_BF16:
-      return launch_t<__nv_bfloat16>(plan, dense, feats, W, out, cin, cout, stream);
+      return launch_t<__nv_bfloat16>(plan, dense, feats, W, out, cin, cout, ep, stream);
     default:
       return SMC_ERR_INVALID;
   }

@@ -96,7 +96,72 @@ struct ConvArgs {
   int n_blocks;  // cout / BN
   int dense;     // 1: K = 1, rows in order, one tap, no plan arrays
   uint64_t wait_ns;
+  const uint16_t* bias;      // [cout] or null: epilogue act(acc + bias) + residual
+  const uint16_t* residual;  // [n][cout] or null
+  int act;                   // enum smc_activation
 };
+
+template <bool BF16>
+__device__ __forceinline__ float half_to_float(uint16_t h) {
+  if constexpr (BF16)
+    return __uint_as_float(uint32_t(h) << 16);
+  else
+    return __half2float(__ushort_as_half(h));
+}
+
+__device__ __forceinline__ float act_apply(float v, int act) {
+  switch (act) {
+    case SMC_ACT_RELU:
+      return fmaxf(v, 0.f);
+    case SMC_ACT_SILU:
+      return v / (1.f + expf(-v));
+    case SMC_ACT_GELU:
+      return 0.5f * v * (1.f + erff(v * 0.7071067811865476f));
+    default:
+      return v;
+  }
+}
+
+// act(acc + bias) + residual on 32 consecutive columns of one output row (in
+// place, fp32), before the one rounding to the output dtype.
+template <bool BF16>
+__device__ __forceinline__ void apply_epilogue(uint32_t (&v)[32], const ConvArgs& a, int64_t row,
+                                               int col) {
+  if (a.bias) {
+    const uint4* b4 = reinterpret_cast<const uint4*>(a.bias + col);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 u = __ldg(b4 + q);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        v[8 * q + 2 * e] = __float_as_uint(__uint_as_float(v[8 * q + 2 * e]) +
+                                           half_to_float<BF16>(uint16_t(w[e] & 0xFFFFu)));
+        v[8 * q + 2 * e + 1] = __float_as_uint(__uint_as_float(v[8 * q + 2 * e + 1]) +
+                                               half_to_float<BF16>(uint16_t(w[e] >> 16)));
+      }
+    }
+  }
+  if (a.act != SMC_ACT_NONE) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(act_apply(__uint_as_float(v[i]), a.act));
+  }
+  if (a.residual) {
+    const uint4* r4 = reinterpret_cast<const uint4*>(a.residual + row * a.cout + col);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 u = r4[q];
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        v[8 * q + 2 * e] = __float_as_uint(__uint_as_float(v[8 * q + 2 * e]) +
+                                           half_to_float<BF16>(uint16_t(w[e] & 0xFFFFu)));
+        v[8 * q + 2 * e + 1] = __float_as_uint(__uint_as_float(v[8 * q + 2 * e + 1]) +
+                                               half_to_float<BF16>(uint16_t(w[e] >> 16)));
+      }
+    }
+  }
+}
 
 // A work item as the scheduler publishes it.
 template <int G>
@@ -559,6 +624,8 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
           tmem_ld_x32(tmem + (uint32_t(quarter * 32) << 16) + (a * G + k) * BN + uint32_t(cc * 32),
                       v);
           if (orow[k] >= 0) {
+            if (args.bias || args.residual || args.act != SMC_ACT_NONE)
+              apply_epilogue<BF16>(v, args, orow[k], it.n0 + cc * 32);
             uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -647,7 +714,7 @@ bool encode_2d(CUtensorMap* map, bool bf16, const void* base, uint64_t cols, uin
 
 template <int BN, int NA, int NW, int G, int WPS, int NQ, bool BF16, int NBUF>
 int launch_cfg(const Plan& plan, bool dense, const void* feats, const void* W, void* out, int cin,
-               int cout, cudaStream_t stream) {
+               int cout, const Epilogue& ep, cudaStream_t stream) {
   constexpr int kWBytes = BN * kBK * 2;
   constexpr int kBars = 4 * NA + 2 * NW + 6 + 2 * kQueue + 2;
   constexpr int kTail = kBars * 8 + (kQueue + 2) * int(sizeof(Item<G>)) + 16;
@@ -690,6 +757,9 @@ int launch_cfg(const Plan& plan, bool dense, const void* feats, const void* W, v
   a.dense = dense ? 1 : 0;
   a.work_counter = plan.work_counter;  // zero since the build; reset by each launch
   a.wait_ns = wait_limit_ns();
+  a.bias = static_cast<const uint16_t*>(ep.bias);
+  a.residual = static_cast<const uint16_t*>(ep.residual);
+  a.act = ep.act;
   const int64_t work = int64_t(a.n_groups) * a.n_blocks;
   const int grid = int(std::min<int64_t>(work, sm_count()));
   kern<<<grid, threads_for(NQ, WPS), kSmem, stream>>>(wmap, fmap, a);
@@ -708,7 +778,7 @@ int group_override() {
 
 template <bool BF16>
 int launch_dtype(const Plan& plan, bool dense, const void* feats, const void* W, void* out,
-                 int cin, int cout, cudaStream_t stream) {
+                 int cin, int cout, const Epilogue& ep, cudaStream_t stream) {
   // Few tiles per SM: one tile per work item, so every SM gets work and no SM
   // runs two heavy tiles back to back.
   const bool small = plan.n_tiles < int64_t(6) * sm_count();
@@ -721,16 +791,22 @@ int launch_dtype(const Plan& plan, bool dense, const void* feats, const void* W,
     const int64_t items2 = (plan.n_tiles + 1) / 2 * (cout / 256);
     if (group_override() == 2 ||
         (group_override() == 0 && !dense && items2 >= 2 * int64_t(sm_count())))
-      return launch_cfg<256, 9, 2, 2, 4, 3, BF16, 1>(plan, dense, feats, W, out, cin, cout, stream);
-    return launch_cfg<256, 9, 2, 1, 4, 3, BF16, 2>(plan, dense, feats, W, out, cin, cout, stream);
+      return launch_cfg<256, 9, 2, 2, 4, 3, BF16, 1>(plan, dense, feats, W, out, cin, cout,
+          ep, stream);
+    return launch_cfg<256, 9, 2, 1, 4, 3, BF16, 2>(plan, dense, feats, W, out, cin, cout,
+        ep, stream);
   }
   if (cout % 128 == 0) {
     if (g1)
-      return launch_cfg<128, 10, 3, 1, 2, 5, BF16, 2>(plan, dense, feats, W, out, cin, cout, stream);
-    return launch_cfg<128, 10, 3, 2, 2, 5, BF16, 2>(plan, dense, feats, W, out, cin, cout, stream);
+      return launch_cfg<128, 10, 3, 1, 2, 5, BF16, 2>(plan, dense, feats, W, out, cin, cout,
+          ep, stream);
+    return launch_cfg<128, 10, 3, 2, 2, 5, BF16, 2>(plan, dense, feats, W, out, cin, cout,
+        ep, stream);
   }
-  if (g1) return launch_cfg<64, 12, 3, 1, 2, 6, BF16, 2>(plan, dense, feats, W, out, cin, cout, stream);
-  return launch_cfg<64, 12, 3, 2, 2, 6, BF16, 2>(plan, dense, feats, W, out, cin, cout, stream);
+  if (g1) return launch_cfg<64, 12, 3, 1, 2, 6, BF16, 2>(plan, dense, feats, W, out, cin, cout,
+          ep, stream);
+  return launch_cfg<64, 12, 3, 2, 2, 6, BF16, 2>(plan, dense, feats, W, out, cin, cout,
+      ep, stream);
 }
 
 }  // namespace
@@ -751,11 +827,12 @@ bool conv_tc_supported(int cin, int cout, int dtype) {
 }
 
 int launch_conv_tc(const Plan& plan, bool dense, const void* feats, const void* W, void* out,
-                   int cin, int cout, int dtype, cudaStream_t stream) {
+                   int cin, int cout, int dtype, const Epilogue& ep, cudaStream_t stream) {
   if (plan.n == 0) return SMC_OK;
   if (!conv_tc_supported(cin, cout, dtype)) return SMC_ERR_UNSUPPORTED;
-  if (dtype == SMC_BF16) return launch_dtype<true>(plan, dense, feats, W, out, cin, cout, stream);
-  return launch_dtype<false>(plan, dense, feats, W, out, cin, cout, stream);
+  if (dtype == SMC_BF16)
+    return launch_dtype<true>(plan, dense, feats, W, out, cin, cout, ep, stream);
+  return launch_dtype<false>(plan, dense, feats, W, out, cin, cout, ep, stream);
 }
 
 }  // namespace smc

@@ -55,6 +55,15 @@ struct Plan {
   int64_t issued_rows_taps = 0;
 };
 
+// Fused epilogue of a convolution: out = act(conv + bias) + residual, each
+// part optional (null pointers, act = SMC_ACT_NONE).  bias [cout] and
+// residual [n][cout] are in the convolution's dtype.
+struct Epilogue {
+  const void* bias = nullptr;
+  const void* residual = nullptr;
+  int act = 0;
+};
+
 // Index build (smc_index.cu).  Returns an smc_status.
 int build_plan(const int32_t* coords, int64_t n, int32_t stride, int64_t table_capacity,
                int32_t order, int32_t lookup, cudaStream_t stream, Plan* plan);
@@ -63,7 +72,7 @@ void free_plan(Plan* plan);
 // Tensor-core convolution (smc_conv_tc.cu).  feats/W/out in f16 or bf16.
 // dense = true runs the K = 1 form (rows in order, one tap, no plan arrays).
 int launch_conv_tc(const Plan& plan, bool dense, const void* feats, const void* W, void* out,
-                   int cin, int cout, int dtype, cudaStream_t stream);
+                   int cin, int cout, int dtype, const Epilogue& ep, cudaStream_t stream);
 bool conv_tc_supported(int cin, int cout, int dtype);
 
 // Stable LSD radix sort of (key, value) pairs by the low `bits` bits of the
@@ -102,6 +111,6 @@ int subdivide2(const int32_t* coords, int64_t n, const void* feats, int c, int d
 
 // CUDA-core convolution (smc_conv_simt.cu): any cin, cout, dtype.
 int launch_conv_simt(const Plan& plan, bool dense, const void* feats, const void* W, void* out,
-                     int cin, int cout, int dtype, cudaStream_t stream);
+                     int cin, int cout, int dtype, const Epilogue& ep, cudaStream_t stream);
 
 }  // namespace smc
