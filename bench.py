@@ -300,16 +300,16 @@ def run_ours(args) -> None:
     stream = torch.cuda.current_stream(dev)
 
     # ---- cold index build (timed separately) ----
-    idx = binding.SubMIndex(coords)  # first build: loads kernels, warms the pool
+    idx = binding.SubMIndex(coords, order=args.order)  # first build: loads kernels, warms the pool
     idx.close()
     build_ms = []
     for _ in range(5):
         torch.cuda.synchronize()
         t0 = time.perf_counter()
-        idx = binding.SubMIndex(coords)
+        idx = binding.SubMIndex(coords, order=args.order)
         build_ms.append((time.perf_counter() - t0) * 1e3)
         idx.close()
-    idx = binding.SubMIndex(coords)
+    idx = binding.SubMIndex(coords, order=args.order)
     pairs3, issued3 = idx.plan_stats()
     slots = issued3 // 128
     # a later layer's input is what the earlier layers of the block produce
@@ -404,7 +404,7 @@ def run_ours(args) -> None:
         "dtype": DTYPE_NAME[w.dtype], "data": "synthetic",
         "config": {"workload": args.workload, "grid": w.grid, "batch": w.batch,
                    "n_voxels": inp.n, "layer": args.layer, "cin": cin, "cout": cout, "K": K,
-                   "occupancy": OCCUPANCY[w.sparsity], "seed": 0,
+                   "occupancy": OCCUPANCY[w.sparsity], "seed": 0, "plan_order": args.order,
                    "l2": "flushed between steps (256 MB write, outside the timed events)",
                    "parallelism": f"replicas x{world}"},
         "conv_ms": conv_ms_max,
@@ -452,6 +452,8 @@ def main(argv=None) -> None:
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="uniform128", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--order", default="mask", choices=["mask", "greedy", "input"],
+                    help="row order of the tile plan (index build option)")
     ap.add_argument("--layer", type=int, default=0,
                     help="layer of the workload to time (resblock64: 0 = 3x3x3 512->512, "
                          "1 = 1x1x1 512->1024)")

@@ -63,7 +63,11 @@ enum smc_dtype { SMC_F32 = 0, SMC_F16 = 1, SMC_BF16 = 2 };
 enum smc_order {
   SMC_ORDER_MASK = 0,  /* rows sorted by (number of active taps, Gray-code rank of the
                           tap mask): default */
-  SMC_ORDER_INPUT = 1  /* rows in input order (ablation) */
+  SMC_ORDER_INPUT = 1, /* rows in input order (ablation) */
+  SMC_ORDER_GREEDY = 2 /* the mask order, then greedy packing inside segments of
+                          16,384 rows: each tile grows by the masks that add the
+                          fewest taps to its union (fewer taps multiplied; a
+                          slower build) */
 };
 
 /* How neighbours are looked up (smc_index_options.lookup); both give the same

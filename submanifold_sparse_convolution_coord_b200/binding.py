@@ -24,7 +24,7 @@ STATUS = {
     -8: "SMC_ERR_TIMEOUT",
 }
 DTYPE_CODE = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
-ORDER_CODE = {"mask": 0, "input": 1}
+ORDER_CODE = {"mask": 0, "input": 1, "greedy": 2}
 LOOKUP_CODE = {"hash": 0, "sort": 1}
 
 # every symbol include/smc.h declares

@@ -111,7 +111,8 @@ int smc_build_index_ex(const int32_t* coords_dev, int64_t n, int32_t stride,
   int32_t order = SMC_ORDER_MASK, lookup = SMC_LOOKUP_HASH;
   if (opts) {
     if (opts->table_capacity < 0 ||
-        (opts->order != SMC_ORDER_MASK && opts->order != SMC_ORDER_INPUT) ||
+        (opts->order != SMC_ORDER_MASK && opts->order != SMC_ORDER_INPUT &&
+         opts->order != SMC_ORDER_GREEDY) ||
         (opts->lookup != SMC_LOOKUP_HASH && opts->lookup != SMC_LOOKUP_SORT))
       return SMC_ERR_INVALID;
     cap = opts->table_capacity;

@@ -190,6 +190,170 @@ k_neighbors_sorted(const int4* __restrict__ coords, int64_t n, int32_t stride,
   }
 }
 
+// ---------------------------------------------------------------------------
+// Greedy tile packing (SMC_ORDER_GREEDY).  The mask-sorted rows are cut into
+// segments of kGreedySeg rows, one CTA each.  Inside a segment, equal masks
+// are contiguous; each tile starts from the first mask with rows left, then
+// alternates (a) taking, in order, every mask whose taps are already in the
+// tile's union, and (b) taking the one mask that adds the fewest new taps
+// (most rows on ties), until 128 rows.  The tensor-core kernel multiplies
+// 128 rows per tap of a tile's union, so fewer union taps is less work.
+// Output: a plan-row permutation with the same tile layout as the sort.
+// ---------------------------------------------------------------------------
+constexpr int kGreedySeg = 16384;   // rows per segment (a multiple of 128)
+constexpr int kGreedyThreads = 512;
+constexpr int kGreedyPer = kGreedySeg / kGreedyThreads;  // distinct masks per thread, at most
+
+// Block-wide exclusive scan of one value per thread (kGreedyThreads threads);
+// returns the prefix, *total gets the sum.
+__device__ __forceinline__ int block_scan(int v, int* total, int* wsum) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < kGreedyThreads / 32 ? wsum[lane] : 0;
+    int wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += t;
+    }
+    if (lane < kGreedyThreads / 32) wsum[lane] = wi - w;  // exclusive warp offsets
+    if (lane == kGreedyThreads / 32 - 1) wsum[32] = wi;
+  }
+  __syncthreads();
+  const int r = wsum[warp] + incl - v;
+  *total = wsum[32];
+  __syncthreads();
+  return r;
+}
+
+// Block-wide minimum of a 64-bit key (kGreedyThreads threads).
+__device__ __forceinline__ unsigned long long block_min(unsigned long long v,
+                                                       unsigned long long* wmin) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if (lane == 0) wmin[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    unsigned long long w = lane < kGreedyThreads / 32 ? wmin[lane] : ~0ull;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) w = min(w, __shfl_xor_sync(0xffffffffu, w, o));
+    if (lane == 0) wmin[32] = w;
+  }
+  __syncthreads();
+  const unsigned long long r = wmin[32];
+  __syncthreads();
+  return r;
+}
+
+__global__ void __launch_bounds__(kGreedyThreads)
+k_greedy_tiles(const int32_t* __restrict__ sorted_rows, const uint32_t* __restrict__ mask,
+               int64_t n, int32_t* __restrict__ perm) {
+  extern __shared__ uint32_t gsm[];
+  uint32_t* u = gsm;                                          // distinct masks, in order
+  uint16_t* live = reinterpret_cast<uint16_t*>(u + kGreedySeg);   // rows left per mask
+  uint16_t* next = live + kGreedySeg;                         // next row to take (segment offset)
+  __shared__ int wsum[33];
+  __shared__ unsigned long long wmin[33];
+  const int64_t base = int64_t(blockIdx.x) * kGreedySeg;
+  const int len = int(n - base < int64_t(kGreedySeg) ? n - base : int64_t(kGreedySeg));
+  const int t0 = threadIdx.x * kGreedyPer;  // this thread's rows, then its distinct masks
+
+  // run-length encode the segment's masks: distinct index of each head row
+  int heads = 0;
+  uint32_t prev = t0 > 0 && t0 < len ? mask[sorted_rows[base + t0 - 1]] : 0u;
+  for (int i = t0; i < t0 + kGreedyPer && i < len; ++i) {
+    const uint32_t m = mask[sorted_rows[base + i]];
+    heads += (i == 0 || m != prev) ? 1 : 0;
+    prev = m;
+  }
+  int d = 0;
+  int q = block_scan(heads, &d, wsum);
+  prev = t0 > 0 && t0 < len ? mask[sorted_rows[base + t0 - 1]] : 0u;
+  for (int i = t0; i < t0 + kGreedyPer && i < len; ++i) {
+    const uint32_t m = mask[sorted_rows[base + i]];
+    if (i == 0 || m != prev) {
+      u[q] = m;
+      next[q] = uint16_t(i);
+      ++q;
+    }
+    prev = m;
+  }
+  __syncthreads();
+  for (int k = t0; k < t0 + kGreedyPer; ++k)
+    if (k < d) live[k] = uint16_t((k + 1 < d ? int(next[k + 1]) : len) - int(next[k]));
+  __syncthreads();
+
+  // take `t` rows of distinct mask k into plan rows out, out + 1, ...
+  auto take = [&](int k, int t, int64_t out) {
+    const int r0 = next[k];
+    for (int j = 0; j < t; ++j) perm[out + j] = sorted_rows[base + r0 + j];
+  };
+
+  int64_t out = base;
+  const int64_t end = base + len;
+  while (out < end) {
+    // a new tile from the first mask with rows left
+    unsigned long long key = ~0ull;
+    for (int k = t0; k < t0 + kGreedyPer && k < d; ++k)
+      if (live[k] > 0) {
+        key = k;
+        break;
+      }
+    key = block_min(key, wmin);
+    uint32_t U = u[key];
+    int fill = 0;
+    bool pick_next = false;  // the first mask is taken by the subset pass below
+    while (fill < kTileRows) {
+      if (pick_next) {
+        // the mask adding the fewest taps to U, most rows on ties, first index
+        unsigned long long best = ~0ull;
+        for (int k = t0; k < t0 + kGreedyPer && k < d; ++k) {
+          if (live[k] == 0) continue;
+          const unsigned add = __popc(u[k] & ~U);
+          const unsigned rows = min(int(live[k]), kTileRows - fill);
+          const unsigned long long kk =
+              (uint64_t(add) << 40) | (uint64_t(kTileRows - rows) << 24) | uint64_t(k);
+          best = min(best, kk);
+        }
+        best = block_min(best, wmin);
+        if (best == ~0ull) break;  // the segment is used up
+        const int k = int(best & 0xFFFFFF);
+        U |= u[k];
+      }
+      pick_next = true;
+      // every mask inside U, in order, until the tile is full
+      int mine = 0;
+      for (int k = t0; k < t0 + kGreedyPer && k < d; ++k)
+        if (live[k] > 0 && (u[k] & ~U) == 0u) mine += live[k];
+      int total = 0;
+      int pre = block_scan(mine, &total, wsum);
+      for (int k = t0; k < t0 + kGreedyPer && k < d; ++k) {
+        if (live[k] == 0 || (u[k] & ~U) != 0u) continue;
+        const int t = max(0, min(int(live[k]), kTileRows - fill - pre));
+        if (t > 0) {
+          take(k, t, out + fill + pre);
+          next[k] = uint16_t(next[k] + t);
+          live[k] = uint16_t(live[k] - t);
+        }
+        pre += live[k] + t;  // this mask's rows before the take, for the next mask
+      }
+      fill = min(kTileRows, fill + total);
+      __syncthreads();
+      if (fill >= kTileRows || out + fill >= end) break;
+    }
+    out += fill;
+  }
+}
+
 // Sort key: popcount in the top 5 bits (so tiles come out lightest to
 // heaviest), then the rank of the 27-bit mask in reflected Gray-code order
 // (the prefix XOR of the mask): consecutive masks in that order differ in one
@@ -527,6 +691,22 @@ int build_plan_impl(const int32_t* coords, int64_t n, int32_t stride, int64_t ta
     if (cudaMemcpyAsync(plan->perm, sc.svals[cur], size_t(n) * sizeof(int32_t),
                         cudaMemcpyDeviceToDevice, s) != cudaSuccess)
       return SMC_ERR_CUDA;
+  } else if (order == SMC_ORDER_GREEDY) {
+    k_sort_keys<<<grid_for(n, 256), 256, 0, s>>>(plan->mask, n, sc.skeys[0], sc.svals[0]);
+    SMC_LAUNCHED();
+    int cur = 0;
+    SMC_TRY(radix_sort(sc.skeys, sc.svals, 0, n, 32, sc.hist, s, &cur));
+    constexpr int kSmem = kGreedySeg * (4 + 2 + 2);
+    static bool attr_set = false;  // a function attribute: idempotent, set on first use
+    if (!attr_set) {
+      if (cudaFuncSetAttribute(k_greedy_tiles, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kSmem) != cudaSuccess)
+        return SMC_ERR_CUDA;
+      attr_set = true;
+    }
+    k_greedy_tiles<<<grid_for(n, kGreedySeg), kGreedyThreads, kSmem, s>>>(sc.svals[cur],
+                                                                          plan->mask, n, plan->perm);
+    SMC_LAUNCHED();
   } else {
     k_iota<<<grid_for(n, 256), 256, 0, s>>>(plan->perm, n);
     SMC_LAUNCHED();

@@ -109,6 +109,47 @@ def test_input_order_plan():
     idx.close()
 
 
+@pytest.mark.parametrize("name", ["uniform64", "uniform128", "resblock64"])
+def test_greedy_order_plan_and_conv(name):
+    """The greedy tile packing: a valid plan (bijection, every pair covered,
+    exact tile masks), fewer issued rows x taps than the mask sort, and the
+    convolution over it matching the oracle on every row."""
+    inp = synth.make_inputs(name)
+    ref = native.neighbor_map(inp.coords)
+    idx, m = _gpu_map(inp.coords, order="greedy")
+    assert np.array_equal(m, ref)
+    _check_plan(idx, ref)
+    sorted_idx, _ = _gpu_map(inp.coords, order="mask")
+    assert idx.plan_stats()[1] <= sorted_idx.plan_stats()[1]
+    sorted_idx.close()
+    W = inp.weights[0]
+    out = idx.forward(inp.feats.to(DEV), W.to(DEV))
+    torch.cuda.synchronize()
+    assert idx.status() == 0
+    want, scale = native.submconv(inp.feats.double().numpy(), W.double().numpy(), ref)
+    from gpu_common import check_conv
+    check_conv(out, want, scale, f"{name} greedy")
+    idx.close()
+
+
+def test_greedy_order_segments_and_edges():
+    """Several 16,384-row segments with a ragged last one, shuffled input,
+    and the small edge cases of the plan."""
+    co, feats, W = synth.random_case(7, 40000, 60, 1, 64, 64, 3, "f16", shuffle=True)
+    ref = native.neighbor_map(co)
+    idx, m = _gpu_map(co, order="greedy")
+    assert np.array_equal(m, ref)
+    _check_plan(idx, ref)
+    idx.close()
+    for case in ("single_voxel", "n129", "two_batches_touching"):
+        coords = _adversarial_cases()[case]
+        idx, m = _gpu_map(coords, order="greedy")
+        r = native.neighbor_map(coords)
+        assert np.array_equal(m, r)
+        _check_plan(idx, r)
+        idx.close()
+
+
 def test_empty_index():
     c = torch.zeros((0, 4), dtype=torch.int32, device=DEV)
     idx = SubMIndex(c)
