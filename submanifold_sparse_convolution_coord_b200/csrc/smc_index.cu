@@ -697,12 +697,16 @@ int build_plan_impl(const int32_t* coords, int64_t n, int32_t stride, int64_t ta
     int cur = 0;
     SMC_TRY(radix_sort(sc.skeys, sc.svals, 0, n, 32, sc.hist, s, &cur));
     constexpr int kSmem = kGreedySeg * (4 + 2 + 2);
-    static bool attr_set = false;  // a function attribute: idempotent, set on first use
-    if (!attr_set) {
+    // the shared-memory limit is a per-device function attribute
+    constexpr int kMaxDev = 64;
+    static bool attr_set[kMaxDev] = {};
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SMC_ERR_CUDA;
+    if (!(dev >= 0 && dev < kMaxDev && attr_set[dev])) {
       if (cudaFuncSetAttribute(k_greedy_tiles, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kSmem) != cudaSuccess)
         return SMC_ERR_CUDA;
-      attr_set = true;
+      if (dev >= 0 && dev < kMaxDev) attr_set[dev] = true;
     }
     k_greedy_tiles<<<grid_for(n, kGreedySeg), kGreedyThreads, kSmem, s>>>(sc.svals[cur],
                                                                           plan->mask, n, plan->perm);
