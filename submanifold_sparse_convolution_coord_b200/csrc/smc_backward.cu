@@ -221,6 +221,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) k_bwd_weight_tc(const BwdArgs 
     const int a_chunks = (cib_w / 64) * 8;           // 16-byte chunks per A row
     constexpr int g_chunks = (BN / 64) * 8;
     bool ok = wt.wait(idx_bar, 0);
+    // A stage is published (copies landed, proxy fence, arrival) once the next
+    // stage's copies are issued, so two stages' copies stay in flight; the
+    // last one after the loop.
+    int pend = -1;
     for (int s = 0; s < n_stages && ok; ++s) {
       const int slot = s % kBwdStages;
       if (!wt.wait(empty0 + 8 * slot, ((s / kBwdStages) & 1) ^ 1)) {
@@ -256,7 +260,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1) k_bwd_weight_tc(const BwdArgs 
         cp_async_16(base + 2 * kBwdAtom + atom * kBwdAtom + row * 128 + ((ch ^ (row & 7)) << 4),
                     src, i >= 0 ? 16u : 0u);
       }
-      cp_async_arrive_noinc(full0 + 8 * slot);
+      cp_async_commit();
+      if (pend >= 0) {
+        cp_async_wait_group<1>();
+        fence_proxy_async_smem();
+        mbar_arrive(full0 + 8 * pend);
+      }
+      pend = slot;
+    }
+    if (ok && pend >= 0) {
+      cp_async_wait_group<0>();
+      fence_proxy_async_smem();
+      mbar_arrive(full0 + 8 * pend);
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == kBwdMmaWarp) {

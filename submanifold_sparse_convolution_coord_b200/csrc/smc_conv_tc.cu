@@ -442,6 +442,21 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
     if (args.dense && wq == 0 && lane == 0) tma_prefetch_map(&fmap);
     uint32_t u = 0, j = 0;
     int last_dense = -1;  // last unit this group TMA-loaded (dense mode)
+    // The unit whose copies this lane issued last and has not yet published:
+    // it is published (copies landed, proxy fence, arrival) after the next
+    // unit's copies are issued, so two units' copies stay in flight, and at
+    // the end of every item, so no unit waits on a later item.
+    int pend = -1;
+    auto publish = [&](bool keep_newest) {
+      if (pend < 0) return;
+      if (keep_newest)
+        cp_async_wait_group<1>();
+      else
+        cp_async_wait_group<0>();
+      fence_proxy_async_smem();
+      mbar_arrive(afull0 + 8 * pend);
+      pend = -1;
+    };
     bool ok = true;
     while (ok) {
       const Item<G> it = next_item(j, true);
@@ -497,10 +512,13 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
               // 128-byte swizzle: chunk c of row r sits at chunk c ^ (r & 7)
               cp_async_16(dst + row * 128 + ((chunk ^ (row & 7)) << 4), src, v[i] >= 0 ? 16u : 0u);
             }
-            cp_async_arrive_noinc(afull0 + 8 * slot);
+            cp_async_commit();
+            publish(true);  // the previous unit: all but this unit's copies have landed
+            pend = int(slot);
           }
         }
       }
+      if (ok) publish(false);
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
     if (last_dense >= 0) {
