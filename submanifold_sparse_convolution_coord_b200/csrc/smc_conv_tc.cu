@@ -238,6 +238,10 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
   // can be two phases behind, and the abort path can tell which of its loads
   // may still be in flight.
   static_assert(NA % NQ == 0, "every A slot is owned by one gather group");
+  // A group publishes a unit only after issuing its next one, which needs a
+  // different slot: with a single slot per group the next unit would wait on
+  // the very slot the unpublished one holds.
+  static_assert(NA / NQ >= 2, "each gather group needs at least two A slots");
   static_assert(NBUF == 1 || NBUF == 2, "accumulator sets");
   constexpr int kWBytes = BN * kBK * 2;          // one W slice
   constexpr int kRowsPerWarp = kTileRows / WPS;  // rows of a unit one gather warp copies
@@ -417,6 +421,9 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
                 ok = false;
                 break;
               }
+              // the gathers' reads of this block (generic proxy) come before the
+              // bulk copy that overwrites it (async proxy)
+              fence_proxy_async_smem();
               const int slot = it.slot0[k] + __popc(it.mask[k] & ((1u << tap) - 1u));
               mbar_arrive_expect_tx(ifull0 + 8 * is, kIdxBytes);
               bulk_load(i_base + is * kIdxBytes, args.gidx + int64_t(slot) * kTileRows, kIdxBytes,
@@ -497,6 +504,9 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
             const int32_t* idx = idx_ring + slot * kTileRows + row0 + rsub;
 #pragma unroll
             for (int i = 0; i < kInstr; ++i) v[i] = idx[4 * i];
+            // the block is refilled by a bulk copy (async proxy) once released:
+            // order these generic-proxy reads before that write
+            fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(iempty0 + 8 * slot);
             got = wt.wait(aempty0 + 8 * slot, ph ^ 1);

@@ -200,7 +200,7 @@ k_neighbors_sorted(const int4* __restrict__ coords, int64_t n, int32_t stride,
 // 128 rows per tap of a tile's union, so fewer union taps is less work.
 // Output: a plan-row permutation with the same tile layout as the sort.
 // ---------------------------------------------------------------------------
-constexpr int kGreedySeg = 16384;   // rows per segment (a multiple of 128)
+constexpr int kGreedySeg = 8192;    // rows per segment (a multiple of 128)
 constexpr int kGreedyThreads = 512;
 constexpr int kGreedyPer = kGreedySeg / kGreedyThreads;  // distinct masks per thread, at most
 
@@ -259,7 +259,8 @@ k_greedy_tiles(const int32_t* __restrict__ sorted_rows, const uint32_t* __restri
                int64_t n, int32_t* __restrict__ perm) {
   extern __shared__ uint32_t gsm[];
   uint32_t* u = gsm;                                          // distinct masks, in order
-  uint16_t* live = reinterpret_cast<uint16_t*>(u + kGreedySeg);   // rows left per mask
+  int32_t* rows = reinterpret_cast<int32_t*>(u + kGreedySeg);    // the segment's sorted rows
+  uint16_t* live = reinterpret_cast<uint16_t*>(rows + kGreedySeg);  // rows left per mask
   uint16_t* next = live + kGreedySeg;                         // next row to take (segment offset)
   __shared__ int wsum[33];
   __shared__ unsigned long long wmin[33];
@@ -267,19 +268,21 @@ k_greedy_tiles(const int32_t* __restrict__ sorted_rows, const uint32_t* __restri
   const int len = int(n - base < int64_t(kGreedySeg) ? n - base : int64_t(kGreedySeg));
   const int t0 = threadIdx.x * kGreedyPer;  // this thread's rows, then its distinct masks
 
+  for (int i = threadIdx.x; i < len; i += kGreedyThreads) rows[i] = sorted_rows[base + i];
+  __syncthreads();
   // run-length encode the segment's masks: distinct index of each head row
   int heads = 0;
-  uint32_t prev = t0 > 0 && t0 < len ? mask[sorted_rows[base + t0 - 1]] : 0u;
+  uint32_t prev = t0 > 0 && t0 < len ? mask[rows[t0 - 1]] : 0u;
   for (int i = t0; i < t0 + kGreedyPer && i < len; ++i) {
-    const uint32_t m = mask[sorted_rows[base + i]];
+    const uint32_t m = mask[rows[i]];
     heads += (i == 0 || m != prev) ? 1 : 0;
     prev = m;
   }
   int d = 0;
   int q = block_scan(heads, &d, wsum);
-  prev = t0 > 0 && t0 < len ? mask[sorted_rows[base + t0 - 1]] : 0u;
+  prev = t0 > 0 && t0 < len ? mask[rows[t0 - 1]] : 0u;
   for (int i = t0; i < t0 + kGreedyPer && i < len; ++i) {
-    const uint32_t m = mask[sorted_rows[base + i]];
+    const uint32_t m = mask[rows[i]];
     if (i == 0 || m != prev) {
       u[q] = m;
       next[q] = uint16_t(i);
@@ -295,7 +298,7 @@ k_greedy_tiles(const int32_t* __restrict__ sorted_rows, const uint32_t* __restri
   // take `t` rows of distinct mask k into plan rows out, out + 1, ...
   auto take = [&](int k, int t, int64_t out) {
     const int r0 = next[k];
-    for (int j = 0; j < t; ++j) perm[out + j] = sorted_rows[base + r0 + j];
+    for (int j = 0; j < t; ++j) perm[out + j] = rows[r0 + j];
   };
 
   int64_t out = base;
@@ -696,7 +699,7 @@ int build_plan_impl(const int32_t* coords, int64_t n, int32_t stride, int64_t ta
     SMC_LAUNCHED();
     int cur = 0;
     SMC_TRY(radix_sort(sc.skeys, sc.svals, 0, n, 32, sc.hist, s, &cur));
-    constexpr int kSmem = kGreedySeg * (4 + 2 + 2);
+    constexpr int kSmem = kGreedySeg * (4 + 4 + 2 + 2);
     // the shared-memory limit is a per-device function attribute
     constexpr int kMaxDev = 64;
     static bool attr_set[kMaxDev] = {};
