@@ -16,7 +16,8 @@
 //               gather index [tile][active tap][128 rows];
 //   5. items    for work items of one and of two consecutive tiles, the
 //               groups in decreasing order of their union's tap count (one
-//               stable radix pass), so the convolution hands out its largest
+//               block-wide stable counting sort, or a radix pass for more
+//               than 49,152 tiles), so the convolution hands out its largest
 //               items first, each written as a 16-byte record (first tile,
 //               tap masks, first gather-index slot) the convolution's
 //               scheduler reads with one load.
@@ -450,6 +451,73 @@ __global__ void k_group_keys(const uint32_t* __restrict__ tile_mask, int64_t n_t
   vals[i] = int32_t(g);
 }
 
+// Work items of G = blockIdx.x + 1 tiles in one block: the same order as
+// k_group_keys + a stable sort + k_item_records (most union taps first; among
+// equal counts the later group first), as a stable counting sort over the 28
+// possible keys, each key a block-wide scan of per-thread counts.  The keys
+// are cached in shared memory (one byte per group, up to kItemSortMax tiles).
+constexpr int kItemSortMax = 49152;  // within the default 48 KB of dynamic shared memory
+
+__global__ void __launch_bounds__(1024)
+k_item_order(const uint32_t* __restrict__ tile_mask, const int32_t* __restrict__ tile_off,
+             int64_t n_tiles, int4* __restrict__ items1, int4* __restrict__ items2) {
+  extern __shared__ uint8_t key_of[];  // [ng]: 27 - tap count, in listing order i
+  __shared__ int wsum[33];
+  const int G = blockIdx.x + 1;
+  int4* items = G == 1 ? items1 : items2;
+  const int ng = int((n_tiles + G - 1) / G);
+  const int per = (ng + 1023) / 1024;
+  const int i0 = threadIdx.x * per, i1 = min(ng, i0 + per);
+  for (int i = i0; i < i1; ++i) {
+    const int64_t g = ng - 1 - i;  // listed from the last group to the first
+    uint32_t u = tile_mask[g * G];
+    if (G == 2 && g * G + 1 < n_tiles) u |= tile_mask[g * G + 1];
+    key_of[i] = uint8_t(kTaps - __popc(u));
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int base = 0;
+  for (int v = 0; v <= kTaps; ++v) {
+    int c = 0;
+    for (int i = i0; i < i1; ++i) c += key_of[i] == v ? 1 : 0;
+    // block-wide exclusive scan of c
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      const int w = wsum[lane];
+      int wi = w;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, wi, o);
+        if (lane >= o) wi += t;
+      }
+      wsum[lane] = wi - w;
+      if (lane == 31) wsum[32] = wi;
+    }
+    __syncthreads();
+    int pos = base + wsum[warp] + incl - c;
+    const int total = wsum[32];
+    for (int i = i0; i < i1; ++i) {
+      if (key_of[i] != v) continue;
+      const int64_t t = int64_t(ng - 1 - i) * G;
+      int4 r;
+      r.x = int(t);
+      r.y = int(tile_mask[t]);
+      r.z = (G == 2 && t + 1 < n_tiles) ? int(tile_mask[t + 1]) : 0;
+      r.w = tile_off[t];
+      items[pos++] = r;
+    }
+    base += total;
+    __syncthreads();
+  }
+}
+
 // Tap-major tile lists (see Plan::tap_tiles), one block per tap.
 __global__ void __launch_bounds__(1024)
 k_tap_count(const uint32_t* __restrict__ tile_mask, int64_t n_tiles, int32_t* __restrict__ count) {
@@ -687,12 +755,14 @@ int build_plan_impl(const int32_t* coords, int64_t n, int32_t stride, int64_t ta
 
   // 3. row order
   if (order == SMC_ORDER_MASK) {
-    k_sort_keys<<<grid_for(n, 256), 256, 0, s>>>(plan->mask, n, sc.skeys[0], sc.svals[0]);
+    // four 8-bit passes end where they started: sort straight into perm
+    int32_t* vals[2] = {plan->perm, sc.svals[1]};
+    k_sort_keys<<<grid_for(n, 256), 256, 0, s>>>(plan->mask, n, sc.skeys[0], vals[0]);
     SMC_LAUNCHED();
     int cur = 0;
-    SMC_TRY(radix_sort(sc.skeys, sc.svals, 0, n, 32, sc.hist, s, &cur));
-    if (cudaMemcpyAsync(plan->perm, sc.svals[cur], size_t(n) * sizeof(int32_t),
-                        cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    SMC_TRY(radix_sort(sc.skeys, vals, 0, n, 32, sc.hist, s, &cur));
+    if (cur != 0 && cudaMemcpyAsync(plan->perm, vals[cur], size_t(n) * sizeof(int32_t),
+                                    cudaMemcpyDeviceToDevice, s) != cudaSuccess)
       return SMC_ERR_CUDA;
   } else if (order == SMC_ORDER_GREEDY) {
     k_sort_keys<<<grid_for(n, 256), 256, 0, s>>>(plan->mask, n, sc.skeys[0], sc.svals[0]);
@@ -737,18 +807,24 @@ int build_plan_impl(const int32_t* coords, int64_t n, int32_t stride, int64_t ta
                                     plan->tap_tiles);
   SMC_LAUNCHED();
 
-  // 5. work items of one and two tiles, most taps first: one stable radix
-  // pass over the (27 - tap count) keys, which are below 256
-  for (int G = 1; G <= 2; ++G) {
-    const int64_t ng = (nt + G - 1) / G;
-    k_group_keys<<<grid_for(ng, 256), 256, 0, s>>>(plan->tile_mask, nt, G, ng, sc.gkeys[0],
-                                                    sc.gvals);
-    int32_t* gv[2] = {sc.gvals, sc.gorder};
-    int gcur = 0;
-    SMC_TRY(radix_sort(sc.gkeys, gv, 0, ng, 8, sc.hist, s, &gcur));
-    k_item_records<<<grid_for(ng, 256), 256, 0, s>>>(gv[gcur], ng, G, plan->tile_mask,
-                                                      plan->tile_off, nt, plan->items[G - 1]);
+  // 5. work items of one and two tiles, most taps first
+  if (nt <= kItemSortMax) {
+    k_item_order<<<2, 1024, size_t(nt), s>>>(plan->tile_mask, plan->tile_off, nt, plan->items[0],
+                                             plan->items[1]);
     SMC_LAUNCHED();
+  } else {
+    // one stable radix pass over the (27 - tap count) keys, below 256
+    for (int G = 1; G <= 2; ++G) {
+      const int64_t ng = (nt + G - 1) / G;
+      k_group_keys<<<grid_for(ng, 256), 256, 0, s>>>(plan->tile_mask, nt, G, ng, sc.gkeys[0],
+                                                      sc.gvals);
+      int32_t* gv[2] = {sc.gvals, sc.gorder};
+      int gcur = 0;
+      SMC_TRY(radix_sort(sc.gkeys, gv, 0, ng, 8, sc.hist, s, &gcur));
+      k_item_records<<<grid_for(ng, 256), 256, 0, s>>>(gv[gcur], ng, G, plan->tile_mask,
+                                                        plan->tile_off, nt, plan->items[G - 1]);
+      SMC_LAUNCHED();
+    }
   }
 
   // the one read-back: status word, plan counters, slot count
