@@ -35,11 +35,11 @@ int elem_bytes(int dtype) {
 // Make the handle's workspace at least `bytes` long, stream-ordered on s.
 int ensure_workspace(smc_index* h, size_t bytes, cudaStream_t s) {
   if (bytes <= h->work_bytes) return SMC_OK;
-  if (h->work) cudaFreeAsync(h->work, s);
+  if (h->work) smc::dev_free(h->work, s);
   h->work = nullptr;
   h->work_bytes = 0;
   bytes = (bytes + 255) & ~size_t(255);
-  if (cudaMallocAsync(&h->work, bytes, s) != cudaSuccess) {
+  if (smc::dev_alloc(&h->work, bytes, s) != cudaSuccess) {
     cudaGetLastError();
     h->work = nullptr;
     return SMC_ERR_OOM;
@@ -286,7 +286,7 @@ void smc_destroy(smc_handle_t h) {
   if (cur != h->device) cudaSetDevice(h->device);
   smc::free_plan(&h->plan);  // waits for the device first
   if (h->work) {
-    cudaFreeAsync(h->work, nullptr);
+    smc::dev_free(h->work, nullptr);
     cudaStreamSynchronize(nullptr);
   }
   if (cur != h->device) cudaSetDevice(cur);

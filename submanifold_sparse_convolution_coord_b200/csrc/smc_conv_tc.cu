@@ -71,10 +71,12 @@ constexpr int kMmaWarp = 1;
 constexpr int kSchedWarp = 6;
 constexpr int kIndexWarp = 7;
 constexpr int kFirstGatherWarp = 8;
-constexpr int kBK = 64;                          // channels per stage (128-byte rows)
-constexpr int kAUnitBytes = kTileRows * kBK * 2;  // one A unit: 128 rows x 64 channels
+constexpr int kBK = 64;                          // channels per sub-chunk (128-byte rows)
+constexpr int kSubBytes = kTileRows * kBK * 2;    // one A sub-tile: 128 rows x 64 channels
 constexpr int kIdxBytes = kTileRows * 4;          // one unit's gather indices
-constexpr int kQueue = 2;                         // published items ahead of the consumers
+// Published items ahead of the consumers: one for 64/128-column tiles (fewer
+// items reserved per SM near the end of a launch), two for 256-column tiles.
+__host__ __device__ constexpr int queue_depth(int bn) { return bn == 256 ? 2 : 1; }
 
 __host__ __device__ constexpr int threads_for(int nq, int wps) {
   return 32 * (kFirstGatherWarp + nq * wps + 1);
@@ -228,7 +230,7 @@ __device__ __forceinline__ uint32_t live_tiles(const Item<G>& it, int tap) {
 // NA: A units in flight (16 KB each), NW: W slices in flight, NQ gather groups
 // of WPS warps, NBUF accumulator sets in tensor memory (2: the epilogue of one
 // item overlaps the MMAs of the next; 1: room for two 256-column tiles).
-template <int BN, int NA, int NW, int G, int WPS, int NQ, bool BF16, int NBUF>
+template <int BN, int NA, int NW, int G, int WPS, int NQ, bool BF16, int NBUF, int KS>
 __global__ void __launch_bounds__(threads_for(NQ, WPS), 1)
 k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap fmap,
           const ConvArgs args) {
@@ -238,12 +240,12 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
   // can be two phases behind, and the abort path can tell which of its loads
   // may still be in flight.
   static_assert(NA % NQ == 0, "every A slot is owned by one gather group");
-  // A group publishes a unit only after issuing its next one, which needs a
-  // different slot: with a single slot per group the next unit would wait on
-  // the very slot the unpublished one holds.
-  static_assert(NA / NQ >= 2, "each gather group needs at least two A slots");
   static_assert(NBUF == 1 || NBUF == 2, "accumulator sets");
-  constexpr int kWBytes = BN * kBK * 2;          // one W slice
+  static_assert(KS == 1 || KS == 2, "64-channel sub-chunks per unit");
+  constexpr int kQueue = queue_depth(BN);
+  constexpr int kAUnitBytes = KS * kSubBytes;    // one A unit: 128 rows x 64 KS channels
+  constexpr int kWBytes = BN * kBK * 2;          // one W sub-slice: 64 input channels x BN
+  constexpr int kWStage = KS * kWBytes;          // the W of one unit
   constexpr int kRowsPerWarp = kTileRows / WPS;  // rows of a unit one gather warp copies
   constexpr int kInstr = kRowsPerWarp / 4;       // a warp copy instruction covers 4 rows
   static_assert(kRowsPerWarp % 4 == 0 && kInstr >= 1, "gather split");
@@ -262,8 +264,8 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* a_ring = smem;                                   // NA x 16 KB
-  uint8_t* w_ring = a_ring + NA * kAUnitBytes;              // NW x kWBytes
-  int32_t* idx_ring = reinterpret_cast<int32_t*>(w_ring + NW * kWBytes);  // NA x 128
+  uint8_t* w_ring = a_ring + NA * kAUnitBytes;              // NW x kWStage
+  int32_t* idx_ring = reinterpret_cast<int32_t*>(w_ring + NW * kWStage);  // NA x 128
   uint64_t* bars = reinterpret_cast<uint64_t*>(idx_ring + NA * kTileRows);
   // barriers: afull[NA] aempty[NA] ifull[NA] iempty[NA] wfull[NW] wempty[NW]
   //           tfull[2] tempty[2] info[2] qfull[Q] qempty[Q] drain[2]
@@ -274,7 +276,7 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kb_per_tap = args.cin / kBK;
+  const int kb_per_tap = args.cin / (kBK * KS);  // units per tap
   const int total_work = args.n_groups * args.n_blocks;
   const uint32_t afull0 = smem_addr(bars);
   const uint32_t aempty0 = afull0 + 8 * NA;
@@ -383,12 +385,14 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
               break;
             }
             const uint32_t full = wfull0 + 8 * ws;
-            mbar_arrive_expect_tx(full, kWBytes);
-            const uint32_t dst = w_base + ws * kWBytes;
+            mbar_arrive_expect_tx(full, kWStage);
+            const uint32_t dst = w_base + ws * kWStage;
 #pragma unroll
-            for (int jj = 0; jj < BN / 64; ++jj)
-              tma_load_2d(dst + jj * (kBK * 128), &wmap, it.n0 + 64 * jj,
-                          tap * args.cin + kb * kBK, full);
+            for (int sub = 0; sub < KS; ++sub)
+#pragma unroll
+              for (int jj = 0; jj < BN / 64; ++jj)
+                tma_load_2d(dst + sub * kWBytes + jj * (kBK * 128), &wmap, it.n0 + 64 * jj,
+                            tap * args.cin + (kb * KS + sub) * kBK, full);
           }
         }
       }
@@ -449,21 +453,6 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
     if (args.dense && wq == 0 && lane == 0) tma_prefetch_map(&fmap);
     uint32_t u = 0, j = 0;
     int last_dense = -1;  // last unit this group TMA-loaded (dense mode)
-    // The unit whose copies this lane issued last and has not yet published:
-    // it is published (copies landed, proxy fence, arrival) after the next
-    // unit's copies are issued, so two units' copies stay in flight, and at
-    // the end of every item, so no unit waits on a later item.
-    int pend = -1;
-    auto publish = [&](bool keep_newest) {
-      if (pend < 0) return;
-      if (keep_newest)
-        cp_async_wait_group<1>();
-      else
-        cp_async_wait_group<0>();
-      fence_proxy_async_smem();
-      mbar_arrive(afull0 + 8 * pend);
-      pend = -1;
-    };
     bool ok = true;
     while (ok) {
       const Item<G> it = next_item(j, true);
@@ -486,7 +475,10 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
                   ok = false;
                 } else {
                   mbar_arrive_expect_tx(afull0 + 8 * slot, kAUnitBytes);
-                  tma_load_2d(dst, &fmap, kb * kBK, (it.tile0 + k) * kTileRows, afull0 + 8 * slot);
+#pragma unroll
+                  for (int sub = 0; sub < KS; ++sub)
+                    tma_load_2d(dst + sub * kSubBytes, &fmap, (kb * KS + sub) * kBK,
+                                (it.tile0 + k) * kTileRows, afull0 + 8 * slot);
                   last_dense = int(my);
                 }
               }
@@ -514,21 +506,25 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
               ok = false;
               break;
             }
-            const uint16_t* src_col = args.feats + kb * kBK + chunk * 8;
+            const uint16_t* src_col = args.feats + kb * (KS * kBK) + chunk * 8;
 #pragma unroll
             for (int i = 0; i < kInstr; ++i) {
               const int row = row0 + 4 * i + rsub;
               const uint16_t* src = v[i] >= 0 ? src_col + int64_t(v[i]) * args.cin : args.feats;
               // 128-byte swizzle: chunk c of row r sits at chunk c ^ (r & 7)
-              cp_async_16(dst + row * 128 + ((chunk ^ (row & 7)) << 4), src, v[i] >= 0 ? 16u : 0u);
+              const uint32_t d = dst + row * 128 + ((chunk ^ (row & 7)) << 4);
+#pragma unroll
+              for (int sub = 0; sub < KS; ++sub)
+                cp_async_16(d + sub * kSubBytes, v[i] >= 0 ? src + sub * kBK : src,
+                            v[i] >= 0 ? 16u : 0u);
             }
-            cp_async_commit();
-            publish(true);  // the previous unit: all but this unit's copies have landed
-            pend = int(slot);
+            // one arrival per lane on the slot's barrier, made by the hardware
+            // once this lane's copies have landed; the MMA warp orders them
+            // before its tensor-core reads with a proxy fence
+            cp_async_arrive_noinc(afull0 + 8 * slot);
           }
         }
       }
-      if (ok) publish(false);
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
     if (last_dense >= 0) {
@@ -580,7 +576,7 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
             ok = false;
             break;
           }
-          const uint64_t bd = bdesc0 + uint64_t(ws) * (kWBytes >> 4);
+          const uint64_t bd = bdesc0 + uint64_t(ws) * (kWStage >> 4);
 #pragma unroll
           for (int k = 0; k < G; ++k) {
             if (!((live >> k) & 1u)) continue;
@@ -592,6 +588,9 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
               ok = false;
               break;
             }
+            // the rows were written by cp.async (generic proxy) or TMA: order
+            // them before the tensor core's (async-proxy) reads
+            if (!args.dense) fence_proxy_async_smem();
             tc_fence_after();
             // descriptors: the start-address field (bits 0-13, 16-byte units)
             // never carries, so byte offsets add to the 64-bit value
@@ -599,8 +598,12 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
             const uint32_t d_tmem = tmem + (a * G + k) * BN;
             const uint32_t acc = (started >> k) & 1u;
 #pragma unroll
-            for (int kk = 0; kk < kBK / 16; ++kk)
-              umma_f16(d_tmem, ad + 2 * kk, bd + (2048 >> 4) * kk, kIdesc, kk != 0 ? 1u : acc);
+            for (int kk = 0; kk < KS * (kBK / 16); ++kk) {
+              const int sub = kk / (kBK / 16), k16 = kk % (kBK / 16);
+              umma_f16(d_tmem, ad + uint64_t(sub) * (kSubBytes >> 4) + 2 * k16,
+                       bd + uint64_t(sub) * (kWBytes >> 4) + (2048 >> 4) * k16, kIdesc,
+                       kk != 0 ? 1u : acc);
+            }
             umma_commit(aempty0 + 8 * slot);
           }
           if (!ok) break;
@@ -740,16 +743,17 @@ bool encode_2d(CUtensorMap* map, bool bf16, const void* base, uint64_t cols, uin
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, int NA, int NW, int G, int WPS, int NQ, bool BF16, int NBUF>
+template <int BN, int NA, int NW, int G, int WPS, int NQ, bool BF16, int NBUF, int KS>
 int launch_cfg(const Plan& plan, bool dense, const void* feats, const void* W, void* out, int cin,
                int cout, const Epilogue& ep, cudaStream_t stream) {
   constexpr int kWBytes = BN * kBK * 2;
+  constexpr int kQueue = queue_depth(BN);
   constexpr int kBars = 4 * NA + 2 * NW + 6 + 2 * kQueue + 2;
   constexpr int kTail = kBars * 8 + (kQueue + 2) * int(sizeof(Item<G>)) + 16;
-  constexpr int kSmem = 1024 + NA * (kAUnitBytes + kIdxBytes) + NW * kWBytes + kTail;
+  constexpr int kSmem = 1024 + NA * (KS * kSubBytes + kIdxBytes) + NW * KS * kWBytes + kTail;
   static_assert(kSmem <= 227 * 1024, "shared memory");
   static_assert(threads_for(NQ, WPS) <= 1024, "threads");
-  auto kern = k_conv_tc<BN, NA, NW, G, WPS, NQ, BF16, NBUF>;
+  auto kern = k_conv_tc<BN, NA, NW, G, WPS, NQ, BF16, NBUF, KS>;
   // the shared-memory limit is a per-device function attribute: set it once
   // on each device this configuration runs on
   constexpr int kMaxDev = 64;
@@ -811,7 +815,7 @@ int launch_dtype(const Plan& plan, bool dense, const void* feats, const void* W,
   // runs two heavy tiles back to back.
   const bool small = plan.n_tiles < int64_t(6) * sm_count();
   const bool g1 = group_override() == 1 || (small && group_override() != 2);
-  //                          BN  NA NW G WPS NQ
+  //                          BN  NA NW G WPS NQ        NBUF KS
   if (cout % 256 == 0) {
     // sparse: two 256-column tiles per item share each W slice (one
     // accumulator set), as long as that leaves at least two items per SM;
@@ -819,21 +823,30 @@ int launch_dtype(const Plan& plan, bool dense, const void* feats, const void* W,
     const int64_t items2 = (plan.n_tiles + 1) / 2 * (cout / 256);
     if (group_override() == 2 ||
         (group_override() == 0 && !dense && items2 >= 2 * int64_t(sm_count())))
-      return launch_cfg<256, 9, 2, 2, 4, 3, BF16, 1>(plan, dense, feats, W, out, cin, cout,
+      return launch_cfg<256, 9, 2, 2, 4, 3, BF16, 1, 1>(plan, dense, feats, W, out, cin, cout,
           ep, stream);
-    return launch_cfg<256, 9, 2, 1, 4, 3, BF16, 2>(plan, dense, feats, W, out, cin, cout,
+    return launch_cfg<256, 9, 2, 1, 4, 3, BF16, 2, 1>(plan, dense, feats, W, out, cin, cout,
         ep, stream);
   }
   if (cout % 128 == 0) {
-    if (g1)
-      return launch_cfg<128, 10, 3, 1, 2, 5, BF16, 2>(plan, dense, feats, W, out, cin, cout,
+    // 128 input channels per unit where Cin allows: half the hand-offs per
+    // multiply of the 64-channel unit
+    if (cin % 128 == 0) {
+      if (g1)
+        return launch_cfg<128, 4, 2, 1, 4, 2, BF16, 2, 2>(plan, dense, feats, W, out, cin, cout,
+            ep, stream);
+      return launch_cfg<128, 4, 2, 2, 4, 2, BF16, 2, 2>(plan, dense, feats, W, out, cin, cout,
           ep, stream);
-    return launch_cfg<128, 10, 3, 2, 2, 5, BF16, 2>(plan, dense, feats, W, out, cin, cout,
+    }
+    if (g1)
+      return launch_cfg<128, 10, 3, 1, 2, 5, BF16, 2, 1>(plan, dense, feats, W, out, cin, cout,
+          ep, stream);
+    return launch_cfg<128, 10, 3, 2, 2, 5, BF16, 2, 1>(plan, dense, feats, W, out, cin, cout,
         ep, stream);
   }
-  if (g1) return launch_cfg<64, 12, 3, 1, 2, 6, BF16, 2>(plan, dense, feats, W, out, cin, cout,
+  if (g1) return launch_cfg<64, 12, 3, 1, 2, 6, BF16, 2, 1>(plan, dense, feats, W, out, cin, cout,
           ep, stream);
-  return launch_cfg<64, 12, 3, 2, 2, 6, BF16, 2>(plan, dense, feats, W, out, cin, cout,
+  return launch_cfg<64, 12, 3, 2, 2, 6, BF16, 2, 1>(plan, dense, feats, W, out, cin, cout,
       ep, stream);
 }
 

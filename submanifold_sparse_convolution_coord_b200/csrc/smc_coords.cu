@@ -168,7 +168,7 @@ int downsample2(const int32_t* coords, int64_t n, const void* feats, int c, int 
   DownScratch d;
   carve_down(cv, &d, n);
   void* mem = nullptr;
-  if (cudaMallocAsync(&mem, cv.off, s) != cudaSuccess) {
+  if (dev_alloc(&mem, cv.off, s) != cudaSuccess) {
     cudaGetLastError();
     return SMC_ERR_OOM;
   }
@@ -220,7 +220,7 @@ int downsample2(const int32_t* coords, int64_t n, const void* feats, int c, int 
            cudaSuccess ||
        cudaStreamSynchronize(s) != cudaSuccess))
     rc = SMC_ERR_CUDA;
-  cudaFreeAsync(mem, s);
+  dev_free(mem, s);
   if (rc == SMC_OK) rc = status_of(h.status);
   if (rc == SMC_OK) *out_n = int64_t(h.m);
   return rc;
@@ -229,7 +229,7 @@ int downsample2(const int32_t* coords, int64_t n, const void* feats, int c, int 
 int subdivide2(const int32_t* coords, int64_t n, const void* feats, int c, int dtype,
                int32_t* out_coords, void* out_feats, cudaStream_t s) {
   int32_t* status = nullptr;
-  if (cudaMallocAsync(reinterpret_cast<void**>(&status), sizeof(int32_t), s) != cudaSuccess) {
+  if (dev_alloc(reinterpret_cast<void**>(&status), sizeof(int32_t), s) != cudaSuccess) {
     cudaGetLastError();
     return SMC_ERR_OOM;
   }
@@ -254,7 +254,7 @@ int subdivide2(const int32_t* coords, int64_t n, const void* feats, int c, int d
       (cudaMemcpyAsync(&h, status, sizeof(int32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
        cudaStreamSynchronize(s) != cudaSuccess))
     rc = SMC_ERR_CUDA;
-  cudaFreeAsync(status, s);
+  dev_free(status, s);
   if (rc == SMC_OK) rc = status_of(h);
   return rc;
 }

@@ -627,6 +627,8 @@ struct BuildCounters {
   int32_t status;
   uint32_t work_counter[63];   // the tensor-core kernel's item counter (+ finished CTAs)
   unsigned long long stats[2];  // useful pairs, issued rows x taps
+  int32_t total_slots;          // copy of tile_off[n_tiles], for the one read-back
+  int32_t pad;
 };
 
 // The plan's arrays in one arena (sizes are upper bounds where they depend on
@@ -712,7 +714,7 @@ int build_plan_impl(const int32_t* coords, int64_t n, int32_t stride, int64_t ta
   Carve pc;
   BuildCounters* ctr = nullptr;
   carve_plan(pc, plan, &ctr);
-  if (cudaMallocAsync(&plan->arena, pc.off, s) != cudaSuccess) {
+  if (dev_alloc(&plan->arena, pc.off, s) != cudaSuccess) {
     cudaGetLastError();
     plan->arena = nullptr;
     return SMC_ERR_OOM;
@@ -727,7 +729,7 @@ int build_plan_impl(const int32_t* coords, int64_t n, int32_t stride, int64_t ta
   Carve scc;
   Scratch sc;
   carve_scratch(scc, &sc, n, nt, cap, sorted);
-  if (cudaMallocAsync(scratch_mem, scc.off, s) != cudaSuccess) {
+  if (dev_alloc(scratch_mem, scc.off, s) != cudaSuccess) {
     cudaGetLastError();
     *scratch_mem = nullptr;
     return SMC_ERR_OOM;
@@ -828,21 +830,15 @@ int build_plan_impl(const int32_t* coords, int64_t n, int32_t stride, int64_t ta
   }
 
   // the one read-back: status word, plan counters, slot count
-  struct {
-    int32_t status;
-    int32_t total;
-    unsigned long long stats[2];
-  } h{};
-  if (cudaMemcpyAsync(&h.status, plan->status, sizeof(int32_t), cudaMemcpyDeviceToHost, s) !=
-          cudaSuccess ||
-      cudaMemcpyAsync(&h.total, plan->tile_off + nt, sizeof(int32_t), cudaMemcpyDeviceToHost, s) !=
-          cudaSuccess ||
-      cudaMemcpyAsync(h.stats, ctr->stats, sizeof(h.stats), cudaMemcpyDeviceToHost, s) !=
-          cudaSuccess ||
+  if (cudaMemcpyAsync(&ctr->total_slots, plan->tile_off + nt, sizeof(int32_t),
+                      cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return SMC_ERR_CUDA;
+  BuildCounters h;
+  if (cudaMemcpyAsync(&h, ctr, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
       cudaStreamSynchronize(s) != cudaSuccess)
     return SMC_ERR_CUDA;
   SMC_TRY(status_from_device(h.status));
-  plan->total_slots = h.total;
+  plan->total_slots = h.total_slots;
   plan->useful_pairs = int64_t(h.stats[0]);
   plan->issued_rows_taps = int64_t(h.stats[1]);
   return SMC_OK;
@@ -857,7 +853,7 @@ void free_plan(Plan* plan) {
   cudaDeviceSynchronize();
   cudaGetLastError();
   if (plan->arena) {
-    cudaFreeAsync(plan->arena, nullptr);
+    dev_free(plan->arena, nullptr);
     cudaStreamSynchronize(nullptr);
   }
   *plan = Plan{};
@@ -868,7 +864,7 @@ int build_plan(const int32_t* coords, int64_t n, int32_t stride, int64_t table_c
   void* scratch = nullptr;
   int rc = build_plan_impl(coords, n, stride, table_capacity, order, lookup, stream, plan,
                            &scratch);
-  if (scratch) cudaFreeAsync(scratch, stream);  // stream-ordered after the build's kernels
+  if (scratch) dev_free(scratch, stream);  // stream-ordered after the build's kernels
   if (rc != SMC_OK) {
     cudaGetLastError();
     cudaStreamSynchronize(stream);

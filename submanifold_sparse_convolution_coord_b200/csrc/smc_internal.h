@@ -55,6 +55,11 @@ struct Plan {
   int64_t issued_rows_taps = 0;
 };
 
+// Stream-ordered device memory from libsmc's own pool on the current device
+// (smc_pool.cu): freed memory stays reserved for the next allocation.
+cudaError_t dev_alloc(void** ptr, size_t bytes, cudaStream_t s);
+cudaError_t dev_free(void* ptr, cudaStream_t s);
+
 // Fused epilogue of a convolution: out = act(conv + bias) + residual, each
 // part optional (null pointers, act = SMC_ACT_NONE).  bias [cout] and
 // residual [n][cout] are in the convolution's dtype.

@@ -102,9 +102,14 @@ __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint3
                : "memory");
 }
 // cp.async writes shared memory through the generic proxy; tcgen05.mma reads
-// it through the async proxy.  A thread publishes rows it copied only after
-// its copies have landed (wait_group) and a generic-to-async proxy fence, and
-// only then arrives on the barrier the MMA waits on.
+// it through the async proxy.  Each copying lane makes one arrival on the
+// unit's barrier that the hardware performs once the lane's earlier copies
+// have landed (noinc: the barrier's expected count already includes it); the
+// thread that waits on that barrier then issues a generic-to-async proxy
+// fence before its tensor-core reads.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;" ::: "memory");
 }
