@@ -14,14 +14,20 @@
 // matmul.
 //
 // Pipeline units.  The taps of an item are walked in a rotated order; each
-// tap is split into Cin / 64 channel chunks ("stages").  A stage needs one W
-// slice W[tap][64 ci][BN] (shared by the group's tiles) and, for every tile of
-// the group that has the tap, one A unit: 128 gathered rows x 64 channels
-// (16 KB).  W slices and A units live in two separate shared-memory rings, so
-// an A unit is refilled as soon as its own MMAs are done, and a tile whose
-// rows have landed is multiplied without waiting for the other tile.
+// tap is split into Cin / (64 KS) channel chunks ("stages"), KS = 2 (128
+// channels) where Cin allows it for 128-column tiles, else 1.  A stage needs
+// one W slice W[tap][64 KS ci][BN] (shared by the group's tiles) and, for
+// every tile of the group that has the tap, one A unit: 128 gathered rows x
+// 64 KS channels (16 KS KB).  W slices and A units live in two separate
+// shared-memory rings, so an A unit is refilled as soon as its own MMAs are
+// done, and a tile whose rows have landed is multiplied without waiting for
+// the other tile.
 //
-// Persistent kernel, one CTA per SM, 8 + NQ * WPS + 1 warps:
+// Work items are dealt to the CTAs statically, in snake order over the
+// longest-first item list, and every role walks its CTA's items itself, so
+// nothing is claimed or handed out at run time.
+//
+// Persistent kernel, one CTA per SM, 7 + NQ * WPS + 1 warps:
 //   warp 0      W loader: lane 0 TMA-loads each stage's W slice (MN-major,
 //               128-byte swizzle) into the W ring;
 //   warp 1      allocates tensor memory; issues the MMAs (M = 128, N = BN,
@@ -32,19 +38,18 @@
 //   warps 2-5   epilogue: tensor memory -> registers -> fp16/bf16 -> global,
 //               overlapping the next item's MMAs when there are two
 //               accumulator sets (NBUF = 2);
-//   warp 6      scheduler: takes items (most taps first) from a global
-//               counter and publishes their tile masks and gather-index
-//               offsets in a two-entry shared-memory queue;
-//   warp 7      index prefetcher: lane 0 bulk-copies the 128 gather indices
+//   warp 6      index prefetcher: lane 0 bulk-copies the 128 gather indices
 //               of each A unit into a ring of index blocks, running up to a
 //               full ring of units ahead of the gathers;
-//   warps 8..   NQ gather groups of WPS warps.  Units are dealt round-robin to
+//   warps 7..   NQ gather groups of WPS warps.  Units are dealt round-robin to
 //               the groups; a group reads its unit's indices from shared
-//               memory and copies the 128 rows with 16-byte cp.async into a
-//               128-byte-swizzled K-major tile (zero-filled for absent
-//               neighbours); each lane's mbarrier arrival fires when its
-//               copies land.  For K = 1 ("dense" mode) the rows are
-//               contiguous and one lane of the group loads them with TMA.
+//               memory and copies the 128 rows with 16-byte cp.async into
+//               128-byte-swizzled K-major tiles (zero-filled for absent
+//               neighbours); each lane's arrival on the unit's barrier is
+//               made by the hardware when its copies land, and the MMA warp
+//               puts a proxy fence between that barrier and its reads.  For
+//               K = 1 ("dense" mode) the rows are contiguous and one lane of
+//               the group loads them with TMA.
 // Every hand-over is an mbarrier.  Every wait is bounded in time; a wait that
 // runs out marks the CTA aborted and sets the status word, and each role then
 // waits (again bounded) for the asynchronous copies and MMAs it issued before
@@ -68,15 +73,11 @@ using namespace ptx;
 
 constexpr int kLoaderWarp = 0;
 constexpr int kMmaWarp = 1;
-constexpr int kSchedWarp = 6;
-constexpr int kIndexWarp = 7;
-constexpr int kFirstGatherWarp = 8;
+constexpr int kIndexWarp = 6;
+constexpr int kFirstGatherWarp = 7;
 constexpr int kBK = 64;                          // channels per sub-chunk (128-byte rows)
 constexpr int kSubBytes = kTileRows * kBK * 2;    // one A sub-tile: 128 rows x 64 channels
 constexpr int kIdxBytes = kTileRows * 4;          // one unit's gather indices
-// Published items ahead of the consumers: one for 64/128-column tiles (fewer
-// items reserved per SM near the end of a launch), two for 256-column tiles.
-__host__ __device__ constexpr int queue_depth(int bn) { return bn == 256 ? 2 : 1; }
 
 __host__ __device__ constexpr int threads_for(int nq, int wps) {
   return 32 * (kFirstGatherWarp + nq * wps + 1);
@@ -88,7 +89,6 @@ struct ConvArgs {
   const int32_t* gidx;     // [slots][128], -1 = absent
   const int32_t* out_row;  // [n_tiles * 128], -1 = padding row
   const int4* items;       // [n_groups] {first tile, mask0, mask1, first slot}, most taps first
-  uint32_t* work_counter;  // [0] next item, [1] CTAs finished; both 0 between launches
   int32_t* status;
   int64_t n;
   int cin;
@@ -165,7 +165,7 @@ __device__ __forceinline__ void apply_epilogue(uint32_t (&v)[32], const ConvArgs
   }
 }
 
-// A work item as the scheduler publishes it.
+// A work item as every role of a CTA decodes it.
 template <int G>
 struct Item {
   int w;         // item number, -1 = no more work
@@ -177,8 +177,23 @@ struct Item {
   int slot0[G];  // first gather-index slot of each tile
 };
 
+// The j-th item of this CTA: items are dealt over the CTAs in snake order
+// (CTA c takes c, 2 P - 1 - c, 2 P + c, ... of the longest-first list, P CTAs),
+// so every CTA gets a similar mix of long and short items and no item has to
+// be claimed at run time.  -1 past the end.
+__device__ __forceinline__ int item_of(uint32_t j, int total) {
+  const int64_t p = gridDim.x, c = blockIdx.x;
+  const int64_t w = int64_t(j) * p + ((j & 1u) ? p - 1 - c : c);
+  return w < total ? int(w) : -1;
+}
+// The 16-byte record of item w (sparse mode), loaded one item ahead of use.
+__device__ __forceinline__ int4 item_record(const ConvArgs& a, int w) {
+  if (w < 0 || a.dense) return make_int4(0, 0, 0, 0);
+  return __ldg(a.items + w / a.n_blocks);
+}
+
 template <int BN, int G>
-__device__ __forceinline__ Item<G> decode_item(const ConvArgs& a, int w) {
+__device__ __forceinline__ Item<G> decode_item(const ConvArgs& a, int w, int4 r) {
   Item<G> it;
   it.w = w;
   const int q = w / a.n_blocks;
@@ -192,7 +207,6 @@ __device__ __forceinline__ Item<G> decode_item(const ConvArgs& a, int w) {
     }
     it.rot = 0;
   } else {
-    const int4 r = __ldg(a.items + q);
     it.tile0 = r.x;
     it.mask[0] = uint32_t(r.y);
     it.slot0[0] = r.w;
@@ -227,9 +241,10 @@ __device__ __forceinline__ uint32_t live_tiles(const Item<G>& it, int tap) {
   return live;
 }
 
-// NA: A units in flight (16 KB each), NW: W slices in flight, NQ gather groups
-// of WPS warps, NBUF accumulator sets in tensor memory (2: the epilogue of one
-// item overlaps the MMAs of the next; 1: room for two 256-column tiles).
+// NA: A units in flight (16 KS KB each), NW: W slices in flight, NQ gather
+// groups of WPS warps, NBUF accumulator sets in tensor memory (2: the epilogue
+// of one item overlaps the MMAs of the next; 1: room for two 256-column
+// tiles), KS: 64-channel sub-chunks per unit.
 template <int BN, int NA, int NW, int G, int WPS, int NQ, bool BF16, int NBUF, int KS>
 __global__ void __launch_bounds__(threads_for(NQ, WPS), 1)
 k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap fmap,
@@ -240,9 +255,13 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
   // can be two phases behind, and the abort path can tell which of its loads
   // may still be in flight.
   static_assert(NA % NQ == 0, "every A slot is owned by one gather group");
+  // The two MMA warps take the even and odd tiles of an item and meet only at
+  // the W ring, so one can run up to NW stages (NW * G units) ahead of the
+  // other.  Its wait on an A slot must never be two phases ahead of the
+  // barrier: a slot is reused every NA units, hence NW * G <= NA.
+  static_assert(NW * G <= NA, "MMA warps drift by at most one A slot phase");
   static_assert(NBUF == 1 || NBUF == 2, "accumulator sets");
   static_assert(KS == 1 || KS == 2, "64-channel sub-chunks per unit");
-  constexpr int kQueue = queue_depth(BN);
   constexpr int kAUnitBytes = KS * kSubBytes;    // one A unit: 128 rows x 64 KS channels
   constexpr int kWBytes = BN * kBK * 2;          // one W sub-slice: 64 input channels x BN
   constexpr int kWStage = KS * kWBytes;          // the W of one unit
@@ -255,23 +274,23 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
   constexpr uint32_t kIdesc = make_idesc(BN, BF16);
   constexpr int kMmaWarp2 = kFirstGatherWarp + NQ * WPS;
   constexpr uint32_t kMmaWarps = 2;
-  // readers of a queue entry (one arrival each): W loader, index prefetcher,
-  // every gather warp, both MMA warps (the epilogue learns each item from MMA
-  // warp 1, one accumulator at a time)
-  constexpr uint32_t kQueueReaders = 1 + 1 + NQ * WPS + kMmaWarps;
 
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
-  uint8_t* a_ring = smem;                                   // NA x 16 KB
+  // The rings start at the beginning of dynamic shared memory (the kernel
+  // has no static shared variables), which the 128-byte swizzle needs
+  // 1024-byte aligned; a launch where it is not reports that and does nothing.
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if ((smem_addr(smem_raw) & 1023u) != 0) {
+    if (threadIdx.x == 0) atomicOr(args.status, kDevLayout);
+    return;
+  }
+  uint8_t* a_ring = smem_raw;                               // NA x kAUnitBytes
   uint8_t* w_ring = a_ring + NA * kAUnitBytes;              // NW x kWStage
   int32_t* idx_ring = reinterpret_cast<int32_t*>(w_ring + NW * kWStage);  // NA x 128
   uint64_t* bars = reinterpret_cast<uint64_t*>(idx_ring + NA * kTileRows);
   // barriers: afull[NA] aempty[NA] ifull[NA] iempty[NA] wfull[NW] wempty[NW]
-  //           tfull[2] tempty[2] info[2] qfull[Q] qempty[Q] drain[2]
-  constexpr int kBars = 4 * NA + 2 * NW + 6 + 2 * kQueue + 2;
-  Item<G>* queue = reinterpret_cast<Item<G>*>(bars + kBars);
-  Item<G>* acc_info = queue + kQueue;  // item held by each accumulator set
+  //           tfull[2] tempty[2] info[2] drain[2]
+  constexpr int kBars = 4 * NA + 2 * NW + 6 + 2;
+  Item<G>* acc_info = reinterpret_cast<Item<G>*>(bars + kBars);  // item of each accumulator set
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_info + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -287,9 +306,7 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
   const uint32_t tfull0 = wempty0 + 8 * NW;
   const uint32_t tempty0 = tfull0 + 16;
   const uint32_t info0 = tempty0 + 16;
-  const uint32_t qfull0 = info0 + 16;
-  const uint32_t qempty0 = qfull0 + 8 * kQueue;
-  const uint32_t drain0 = qempty0 + 8 * kQueue;
+  const uint32_t drain0 = info0 + 16;
   const uint32_t a_base = smem_addr(a_ring);
   const uint32_t w_base = smem_addr(w_ring);
   const uint32_t i_base = smem_addr(idx_ring);
@@ -313,10 +330,6 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
       mbar_init(info0 + 8 * a, 1);
       mbar_init(drain0 + 8 * a, 1);
     }
-    for (int q = 0; q < kQueue; ++q) {
-      mbar_init(qfull0 + 8 * q, 1);
-      mbar_init(qempty0 + 8 * q, kQueueReaders);
-    }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -327,53 +340,32 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
   const uint32_t tmem = *tmem_slot;
   const Waits wt{abort_flag, args.status, args.wait_ns};
 
-  // Next item from the queue; every reader (a warp, or one thread) reads each
-  // entry once and releases it with one arrival.  warp_wide: all 32 lanes read
-  // and lane 0 releases after the warp has read.  Returns w = -1 at the end or
-  // when the CTA aborts.
-  auto next_item = [&](uint32_t& j, bool warp_wide) -> Item<G> {
+  // Every role walks the CTA's items itself, in the same order: next_item
+  // decodes the j-th item from the record loaded by the previous call and
+  // starts the load of the following record.  w = -1 after the last item.
+  auto next_item = [&](uint32_t& j, int4& rec) -> Item<G> {
     Item<G> it;
-    const uint32_t q = j % kQueue;
-    bool ok = wt.wait(qfull0 + 8 * q, (j / kQueue) & 1);
-    if (warp_wide) ok = __all_sync(0xffffffffu, ok);
-    if (!ok) {
+    const int w = item_of(j, total_work);
+    if (w < 0) {
       it.w = -1;
       return it;
     }
-    it = queue[q];
-    if (warp_wide) __syncwarp();
-    if (!warp_wide || lane == 0) mbar_arrive(qempty0 + 8 * q);
+    it = decode_item<BN, G>(args, w, rec);
     ++j;
+    rec = item_record(args, item_of(j, total_work));
     return it;
   };
+  auto first_record = [&]() { return item_record(args, item_of(0, total_work)); };
 
-  if (warp == kSchedWarp) {
-    // ---------------- scheduler ----------------
-    for (uint32_t j = 0;; ++j) {
-      const uint32_t q = j % kQueue;
-      int w = -2;  // -2: aborted, the entry may still be read and is left alone
-      if (lane == 0 && wt.wait(qempty0 + 8 * q, ((j / kQueue) & 1) ^ 1)) {
-        const uint32_t t = atomicAdd(args.work_counter, 1u);
-        w = t < uint32_t(total_work) ? int(t) : -1;
-        Item<G> it;
-        if (w >= 0)
-          it = decode_item<BN, G>(args, w);
-        else
-          it.w = -1;
-        queue[q] = it;
-        mbar_arrive(qfull0 + 8 * q);  // release: publishes the entry
-      }
-      w = __shfl_sync(0xffffffffu, w, 0);
-      if (w < 0) break;
-    }
-  } else if (warp == kLoaderWarp) {
+  if (warp == kLoaderWarp) {
     // ---------------- W loader ----------------
     if (lane == 0) {
       tma_prefetch_map(&wmap);
       uint32_t s = 0, j = 0;
+      int4 rec = first_record();
       bool ok = true;
       while (ok) {
-        const Item<G> it = next_item(j, false);
+        const Item<G> it = next_item(j, rec);
         if (it.w < 0) break;
         uint32_t rem = rotate_taps(it.all, it.rot);
         while (rem && ok) {
@@ -407,9 +399,10 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
     // ---------------- index prefetcher ----------------
     if (lane == 0) {
       uint32_t u = 0, j = 0;
+      int4 rec = first_record();
       bool ok = true;
       while (ok) {
-        const Item<G> it = next_item(j, false);
+        const Item<G> it = next_item(j, rec);
         if (it.w < 0) break;
         if (args.dense) continue;  // K = 1 has no gather index
         uint32_t rem = rotate_taps(it.all, it.rot);
@@ -452,10 +445,11 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
     const int row0 = kRowsPerWarp * wq;
     if (args.dense && wq == 0 && lane == 0) tma_prefetch_map(&fmap);
     uint32_t u = 0, j = 0;
+    int4 rec = first_record();
     int last_dense = -1;  // last unit this group TMA-loaded (dense mode)
     bool ok = true;
     while (ok) {
-      const Item<G> it = next_item(j, true);
+      const Item<G> it = next_item(j, rec);
       if (it.w < 0) break;
       uint32_t rem = rotate_taps(it.all, it.rot);
       while (rem && ok) {
@@ -542,11 +536,12 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
     // converged; one elected lane issues.
     const uint32_t mine = warp == kMmaWarp ? 0u : 1u;  // this warp's tiles: k % 2 == mine
     uint32_t u = 0, s = 0, j = 0, acc_iter = 0;
+    int4 rec = first_record();
     bool ok = true;
     const uint64_t adesc0 = desc_a_kmajor(a_base);
     const uint64_t bdesc0 = desc_b_mnmajor(w_base, kBK * 128);
     while (ok) {
-      const Item<G> it = next_item(j, true);
+      const Item<G> it = next_item(j, rec);
       const uint32_t a = acc_iter % NBUF;
       const uint32_t use = acc_iter / NBUF;  // earlier uses of accumulator set a
       const bool free = wt.wait(tempty0 + 8 * a, (use & 1) ^ 1);
@@ -682,15 +677,6 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
-  // The last CTA to finish resets the item counter for the next launch (every
-  // CTA's last atomicAdd on it happened before it got here).
-  if (threadIdx.x == 0) {
-    __threadfence();
-    if (atomicAdd(args.work_counter + 1, 1u) == gridDim.x - 1) {
-      atomicExch(args.work_counter, 0u);
-      atomicExch(args.work_counter + 1, 0u);
-    }
-  }
 }
 
 // ----------------------------------------------------------------------------
@@ -747,10 +733,9 @@ template <int BN, int NA, int NW, int G, int WPS, int NQ, bool BF16, int NBUF, i
 int launch_cfg(const Plan& plan, bool dense, const void* feats, const void* W, void* out, int cin,
                int cout, const Epilogue& ep, cudaStream_t stream) {
   constexpr int kWBytes = BN * kBK * 2;
-  constexpr int kQueue = queue_depth(BN);
-  constexpr int kBars = 4 * NA + 2 * NW + 6 + 2 * kQueue + 2;
-  constexpr int kTail = kBars * 8 + (kQueue + 2) * int(sizeof(Item<G>)) + 16;
-  constexpr int kSmem = 1024 + NA * (KS * kSubBytes + kIdxBytes) + NW * KS * kWBytes + kTail;
+  constexpr int kBars = 4 * NA + 2 * NW + 6 + 2;
+  constexpr int kTail = kBars * 8 + 2 * int(sizeof(Item<G>)) + 16;
+  constexpr int kSmem = NA * (KS * kSubBytes + kIdxBytes) + NW * KS * kWBytes + kTail;
   static_assert(kSmem <= 227 * 1024, "shared memory");
   static_assert(threads_for(NQ, WPS) <= 1024, "threads");
   auto kern = k_conv_tc<BN, NA, NW, G, WPS, NQ, BF16, NBUF, KS>;
@@ -787,7 +772,6 @@ int launch_cfg(const Plan& plan, bool dense, const void* feats, const void* W, v
   a.n_blocks = cout / BN;
   a.n_groups = int((plan.n_tiles + G - 1) / G);
   a.dense = dense ? 1 : 0;
-  a.work_counter = plan.work_counter;  // zero since the build; reset by each launch
   a.wait_ns = wait_limit_ns();
   a.bias = static_cast<const uint16_t*>(ep.bias);
   a.residual = static_cast<const uint16_t*>(ep.residual);

@@ -23,6 +23,7 @@ constexpr int32_t kDevDuplicate = 1;
 constexpr int32_t kDevRange = 2;
 constexpr int32_t kDevTableFull = 4;
 constexpr int32_t kDevTimeout = 8;
+constexpr int32_t kDevLayout = 16;  // a kernel found its shared memory misaligned
 
 struct Plan {
   void* arena = nullptr;       // one device allocation holding every array below
