@@ -43,9 +43,14 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 DTYPE_NAME = {"f16": "f16", "bf16": "bf16", "f32": "f32"}
 # dram__bytes_read.sum + dram__bytes_write.sum of one convolution launch of the
-# current kernel, per (workload, layer), from an ncu capture of that launch
-# (bytes).  Workloads not captured with the current kernel report null.
-NCU_TRAFFIC: dict = {}
+# current kernel, per (workload, layer, plan order), from an ncu capture of that
+# launch (bytes; profiles/k_conv_tc_*.md).  Cases not captured with the current
+# kernel report null.
+NCU_TRAFFIC: dict = {
+    ("uniform128", 0, "greedy"): 64478208 + 15020544,
+    ("resblock64", 0, "greedy"): 97104384 + 30331136,
+    ("uniform64", 0, "greedy"): 4840192 + 0,
+}
 # fp32 features run on the CUDA cores with fp64 accumulation: the ALU bound is
 # the fp64 FMA rate, 148 SMs x 64 fp64 lanes x 2 FLOP x 1.965 GHz.
 FP64_ALU_TFLOPS = 148 * 64 * 2 * 1.965e9 / 1e12
@@ -138,31 +143,36 @@ OCCUPANCY = {
 }
 
 
-def index_build_bytes(n: int, slots: int) -> int:
-    """Algorithmic HBM bytes of one index build with the mask-ordered plan.
+def index_build_bytes(n: int, slots: int, order: str = "mask") -> int:
+    """Algorithmic HBM bytes of one index build.
 
     Per voxel: the insert reads 16 B of coordinates and writes a 12 B key and
     value; the neighbour query reads the coordinates again and writes the
     108 B map row and the 4 B mask; the sort builds 8 B key/value pairs from
     the mask and runs four 8-bit passes, each reading the digit (4 B) and
-    moving the pair (8 B in, 8 B out); the permutation is copied (4 B + 4 B);
-    the tile pass reads permutation and mask (8 B), the gather pass the
-    permutation (4 B) and writes the output-row map (4 B).  The hash table is
-    initialised (8 B keys per slot) and read once (12 B per slot); every
-    active slot of a tile reads 128 neighbour entries and writes 128 gather
-    indices.  Table capacity is the power of two at or above 2 n, at least 64.
+    moving the pair (8 B in, 8 B out), the last one straight into the
+    permutation; the greedy order then reads each sorted row and its mask and
+    writes the permutation (12 B); the tile pass reads permutation and mask
+    (8 B), the gather pass the permutation (4 B) and writes the output-row map
+    (4 B).  The hash table is initialised (8 B keys per slot) and read once
+    (12 B per slot); every active slot of a tile reads 128 neighbour entries
+    and writes 128 gather indices.  Table capacity is the power of two at or
+    above 2 n, at least 64.
     """
     cap = 64
     while cap < 2 * n:
         cap <<= 1
-    per_voxel = (16 + 12) + (16 + 108 + 4) + (12 + 4 * 20) + 8 + (8 + 4 + 4)
+    per_voxel = (16 + 12) + (16 + 108 + 4) + (12 + 4 * 20) + (8 + 4 + 4)
+    if order == "greedy":
+        per_voxel += 12
     return n * per_voxel + cap * (8 + 12) + slots * 128 * (4 + 4)
 
 
-def index_build_summary(n: int, slots: int, build_ms: float, hbm_peak: float) -> dict:
+def index_build_summary(n: int, slots: int, build_ms: float, hbm_peak: float,
+                        order: str = "mask") -> dict:
     """Bandwidth view of the index build: algorithmic bytes over the host-timed
     build (which includes device allocation and the status read-back)."""
-    b = index_build_bytes(n, slots)
+    b = index_build_bytes(n, slots, order)
     gbs = b / (build_ms * 1e-3) / 1e9 if build_ms > 0 else None
     return {"ms": build_ms, "timing": "host wall clock, includes allocation and status read-back",
             "algorithmic_bytes": b, "gbs": gbs,
@@ -410,13 +420,14 @@ def run_ours(args) -> None:
         "conv_ms": conv_ms_max,
         "conv_ms_p50": float(np.median(per)),
         "index_build_ms": float(np.median(build_ms)),
-        "index_build": index_build_summary(inp.n, slots, float(np.median(build_ms)), hbm_peak),
+        "index_build": index_build_summary(inp.n, slots, float(np.median(build_ms)), hbm_peak,
+                                           args.order),
         "useful_pairs": pairs, "issued_rows_taps": issued if w.dtype != "f32" else None,
         "useful_fraction": (pairs / issued if issued else None) if w.dtype != "f32" else None,
         "roofline": {"bound": "tensor" if w.dtype != "f32" else "alu", "achieved": achieved,
                      "peak": peak if w.dtype != "f32" else FP64_ALU_TFLOPS, "unit": "TFLOP/s",
                      "frac": achieved / (peak if w.dtype != "f32" else FP64_ALU_TFLOPS),
-                     "traffic": NCU_TRAFFIC.get((args.workload, args.layer)),
+                     "traffic": NCU_TRAFFIC.get((args.workload, args.layer, args.order)),
                      "peak_source": (f"bf16 dense burst, {peak_kind} (fp16 assumed equal)"
                                      if w.dtype != "f32" else
                                      "fp64 FMA: 148 SMs x 64 lanes x 2 x 1.965 GHz"),
@@ -452,7 +463,7 @@ def main(argv=None) -> None:
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="uniform128", choices=sorted(synth.WORKLOADS))
-    ap.add_argument("--order", default="mask", choices=["mask", "greedy", "input"],
+    ap.add_argument("--order", default="greedy", choices=["mask", "greedy", "input"],
                     help="row order of the tile plan (index build option)")
     ap.add_argument("--layer", type=int, default=0,
                     help="layer of the workload to time (resblock64: 0 = 3x3x3 512->512, "

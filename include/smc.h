@@ -65,7 +65,7 @@ enum smc_order {
                           tap mask): default */
   SMC_ORDER_INPUT = 1, /* rows in input order (ablation) */
   SMC_ORDER_GREEDY = 2 /* the mask order, then greedy packing inside segments of
-                          8,192 rows: each tile grows by the masks that add the
+                          1,024 rows: each tile grows by the masks that add the
                           fewest taps to its union (fewer taps multiplied; a
                           slower build) */
 };

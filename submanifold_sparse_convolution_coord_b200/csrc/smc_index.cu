@@ -201,8 +201,8 @@ k_neighbors_sorted(const int4* __restrict__ coords, int64_t n, int32_t stride,
 // 128 rows per tap of a tile's union, so fewer union taps is less work.
 // Output: a plan-row permutation with the same tile layout as the sort.
 // ---------------------------------------------------------------------------
-constexpr int kGreedySeg = 8192;    // rows per segment (a multiple of 128)
-constexpr int kGreedyThreads = 512;
+constexpr int kGreedySeg = 1024;    // rows per segment (a multiple of 128)
+constexpr int kGreedyThreads = 256;
 constexpr int kGreedyPer = kGreedySeg / kGreedyThreads;  // distinct masks per thread, at most
 
 // Block-wide exclusive scan of one value per thread (kGreedyThreads threads);

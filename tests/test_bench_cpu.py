@@ -18,9 +18,11 @@ def test_conv_bytes_uniform128():
 
 def test_index_build_bytes_counts_each_part():
     n, slots = 209715, 13943
-    per_voxel = 28 + 128 + 92 + 8 + 16
+    per_voxel = 28 + 128 + 92 + 16
     cap = 1 << 19  # smallest power of two >= 2 n
     assert bench.index_build_bytes(n, slots) == n * per_voxel + cap * 20 + slots * 1024
+    # the greedy order adds one read of each sorted row and mask and the permutation write
+    assert bench.index_build_bytes(n, slots, "greedy") - bench.index_build_bytes(n, slots) == 12 * n
     # the table never drops below 64 slots, and every part grows with its input
     assert bench.index_build_bytes(0, 0) == 64 * 20
     assert bench.index_build_bytes(n + 1, slots) > bench.index_build_bytes(n, slots)

@@ -133,7 +133,7 @@ def test_greedy_order_plan_and_conv(name):
 
 
 def test_greedy_order_segments_and_edges():
-    """Several 16,384-row segments with a ragged last one, shuffled input,
+    """Many 1,024-row segments with a ragged last one, shuffled input,
     and the small edge cases of the plan."""
     co, feats, W = synth.random_case(7, 40000, 60, 1, 64, 64, 3, "f16", shuffle=True)
     ref = native.neighbor_map(co)
