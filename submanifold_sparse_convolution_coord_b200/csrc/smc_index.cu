@@ -5,9 +5,10 @@
 // is what made the layer compute-bound), built once per coordinate set:
 //
 //   1. insert   every voxel's packed key (b:15 | x:16 | y:16 | z:16 bits) into
-//               an open-addressing table (linear probing, SplitMix64 mixer);
-//   2. query    the 27 neighbours c + stride*d of every voxel -> int32 map
-//               [n][27] (-1 = absent) and a 27-bit tap mask per voxel;
+//               an open-addressing table (linear probing, Fibonacci hashing);
+//   2. query    the 27 neighbours c + stride*d of every voxel (one warp per
+//               voxel, one lane per tap) -> int32 map [n][27] (-1 = absent)
+//               and a 27-bit tap mask per voxel;
 //   3. order    rows by (popcount(mask), Gray-code rank of mask) with a stable
 //               LSD radix sort, so a 128-row tile holds voxels whose active
 //               taps coincide;
@@ -40,12 +41,15 @@ struct __align__(16) Slot {
   int32_t pad;
 };
 
-// SplitMix64 output mixer (Steele, Lea and Flood, "Fast splittable
-// pseudorandom number generators", OOPSLA 2014).
-__device__ __forceinline__ uint64_t mix64(uint64_t z) {
-  z = (z ^ (z >> 30)) * 0xbf58476d1ce4e5b9ull;
-  z = (z ^ (z >> 27)) * 0x94d049bb133111ebull;
-  return z ^ (z >> 31);
+// Fibonacci (multiplicative) hashing, Knuth, The Art of Computer Programming
+// vol. 3, section 6.4: a table of 2^b slots takes the top b bits of
+// key * 2^64 / phi.  The hash is linear in the key, and a neighbour's packed
+// key is the voxel's key plus a per-offset constant (when every coordinate
+// stays in range), so the query computes one product per voxel and adds a
+// per-offset product for each of the 27 taps.
+constexpr uint64_t kFib = 0x9E3779B97F4A7C15ull;
+__device__ __forceinline__ uint64_t hash_slot(uint64_t prod, int shift) {
+  return shift >= 64 ? 0ull : prod >> shift;  // shift = 64 - b (a one-slot table has b = 0)
 }
 
 __device__ __forceinline__ uint64_t pack_key(int64_t b, int64_t x, int64_t y, int64_t z) {
@@ -55,7 +59,7 @@ __device__ __forceinline__ uint64_t pack_key(int64_t b, int64_t x, int64_t y, in
 __device__ __forceinline__ bool axis_ok(int64_t v) { return v >= 0 && v < kMaxAxis; }
 
 __global__ void k_insert(const int4* __restrict__ coords, int64_t n, Slot* table,
-                         uint64_t cap_mask, int32_t* status) {
+                         uint64_t cap_mask, int shift, int32_t* status) {
   const int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
   if (i >= n) return;
   const int4 c = coords[i];
@@ -64,7 +68,7 @@ __global__ void k_insert(const int4* __restrict__ coords, int64_t n, Slot* table
     return;
   }
   const uint64_t key = pack_key(c.x, c.y, c.z, c.w);
-  uint64_t slot = mix64(key) & cap_mask;
+  uint64_t slot = hash_slot(key * kFib, shift);
   for (uint64_t probe = 0; probe <= cap_mask; ++probe) {
     const unsigned long long prev =
         atomicCAS(&table[slot].key, (unsigned long long)kEmptyKey, (unsigned long long)key);
@@ -81,30 +85,30 @@ __global__ void k_insert(const int4* __restrict__ coords, int64_t n, Slot* table
   atomicOr(status, kDevTableFull);
 }
 
-// 32 voxels per block, one thread per (voxel, tap): the map is written with
-// consecutive threads on consecutive words.
-constexpr int kNbrVoxels = 32;
-constexpr int kNbrThreads = kNbrVoxels * kTaps;  // 864
+// One warp per voxel, lane k < 27 looks up tap k: the map row is written by
+// consecutive lanes and the tap mask is the warp's ballot.
+constexpr int kNbrWarps = 8;
 
-__global__ void __launch_bounds__(kNbrThreads)
+__global__ void __launch_bounds__(kNbrWarps * 32)
 k_neighbors(const int4* __restrict__ coords, int64_t n, int32_t stride,
-            const Slot* __restrict__ table, uint64_t cap_mask, int32_t* __restrict__ nbr,
-            uint32_t* __restrict__ mask) {
-  __shared__ uint32_t smask[kNbrVoxels];
-  if (threadIdx.x < kNbrVoxels) smask[threadIdx.x] = 0;
-  __syncthreads();
-  const int local = threadIdx.x / kTaps;
-  const int k = threadIdx.x - local * kTaps;
-  const int64_t i = blockIdx.x * int64_t(kNbrVoxels) + local;
-  if (i < n) {
-    const int4 c = coords[i];
-    const int64_t x = int64_t(c.y) + int64_t(stride) * (k / 9 - 1);
-    const int64_t y = int64_t(c.z) + int64_t(stride) * ((k / 3) % 3 - 1);
-    const int64_t z = int64_t(c.w) + int64_t(stride) * (k % 3 - 1);
-    int32_t found = -1;
+            const Slot* __restrict__ table, uint64_t cap_mask, int shift,
+            int32_t* __restrict__ nbr, uint32_t* __restrict__ mask) {
+  const int lane = threadIdx.x & 31;
+  const int64_t i = blockIdx.x * int64_t(kNbrWarps) + (threadIdx.x >> 5);
+  if (i >= n) return;  // warp-uniform
+  const int k = lane < kTaps ? lane : 0;
+  const int64_t sx = int64_t(stride) * (k / 9 - 1);
+  const int64_t sy = int64_t(stride) * ((k / 3) % 3 - 1);
+  const int64_t sz = int64_t(stride) * (k % 3 - 1);
+  // the tap's key offset (sx, sy, sz in the x, y, z fields), two's complement
+  const uint64_t dprod = uint64_t(sx * 4294967296ll + sy * 65536ll + sz) * kFib;
+  const int4 c = coords[i];
+  int32_t found = -1;
+  if (lane < kTaps) {
+    const int64_t x = int64_t(c.y) + sx, y = int64_t(c.z) + sy, z = int64_t(c.w) + sz;
     if (axis_ok(x) && axis_ok(y) && axis_ok(z)) {
       const uint64_t key = pack_key(c.x, x, y, z);
-      uint64_t slot = mix64(key) & cap_mask;
+      uint64_t slot = hash_slot(pack_key(c.x, c.y, c.z, c.w) * kFib + dprod, shift);
       for (uint64_t probe = 0; probe <= cap_mask; ++probe) {
         const Slot e = table[slot];
         if (e.key == key) {
@@ -115,14 +119,10 @@ k_neighbors(const int4* __restrict__ coords, int64_t n, int32_t stride,
         slot = (slot + 1) & cap_mask;
       }
     }
-    nbr[i * kTaps + k] = found;
-    if (found >= 0) atomicOr(&smask[local], 1u << k);
+    nbr[i * kTaps + lane] = found;
   }
-  __syncthreads();
-  if (threadIdx.x < kNbrVoxels) {
-    const int64_t ii = blockIdx.x * int64_t(kNbrVoxels) + threadIdx.x;
-    if (ii < n) mask[ii] = smask[threadIdx.x];
-  }
+  const uint32_t m = __ballot_sync(0xffffffffu, found >= 0) & ((1u << kTaps) - 1u);
+  if (lane == 0) mask[i] = m;
 }
 
 // ---------------------------------------------------------------------------
@@ -153,22 +153,20 @@ __global__ void k_sorted_dups(const unsigned long long* __restrict__ keys, int64
   if (i >= 1 && i < n && keys[i] == keys[i - 1]) atomicOr(status, kDevDuplicate);
 }
 
-__global__ void __launch_bounds__(kNbrThreads)
+__global__ void __launch_bounds__(kNbrWarps * 32)
 k_neighbors_sorted(const int4* __restrict__ coords, int64_t n, int32_t stride,
                    const unsigned long long* __restrict__ skeys, const int32_t* __restrict__ svals,
                    int32_t* __restrict__ nbr, uint32_t* __restrict__ mask) {
-  __shared__ uint32_t smask[kNbrVoxels];
-  if (threadIdx.x < kNbrVoxels) smask[threadIdx.x] = 0;
-  __syncthreads();
-  const int local = threadIdx.x / kTaps;
-  const int k = threadIdx.x - local * kTaps;
-  const int64_t i = blockIdx.x * int64_t(kNbrVoxels) + local;
-  if (i < n) {
-    const int4 c = coords[i];
+  const int lane = threadIdx.x & 31;
+  const int64_t i = blockIdx.x * int64_t(kNbrWarps) + (threadIdx.x >> 5);
+  if (i >= n) return;  // warp-uniform
+  const int k = lane < kTaps ? lane : 0;
+  const int4 c = coords[i];
+  int32_t found = -1;
+  if (lane < kTaps) {
     const int64_t x = int64_t(c.y) + int64_t(stride) * (k / 9 - 1);
     const int64_t y = int64_t(c.z) + int64_t(stride) * ((k / 3) % 3 - 1);
     const int64_t z = int64_t(c.w) + int64_t(stride) * (k % 3 - 1);
-    int32_t found = -1;
     if (axis_ok(x) && axis_ok(y) && axis_ok(z)) {
       const unsigned long long key = pack_key(c.x, x, y, z);
       int64_t lo = 0, hi = n;  // first position with skeys[pos] >= key
@@ -181,14 +179,10 @@ k_neighbors_sorted(const int4* __restrict__ coords, int64_t n, int32_t stride,
       }
       if (lo < n && skeys[lo] == key) found = svals[lo];
     }
-    nbr[i * kTaps + k] = found;
-    if (found >= 0) atomicOr(&smask[local], 1u << k);
+    nbr[i * kTaps + lane] = found;
   }
-  __syncthreads();
-  if (threadIdx.x < kNbrVoxels) {
-    const int64_t ii = blockIdx.x * int64_t(kNbrVoxels) + threadIdx.x;
-    if (ii < n) mask[ii] = smask[threadIdx.x];
-  }
+  const uint32_t m = __ballot_sync(0xffffffffu, found >= 0) & ((1u << kTaps) - 1u);
+  if (lane == 0) mask[i] = m;
 }
 
 // ---------------------------------------------------------------------------
@@ -596,6 +590,12 @@ __global__ void k_item_records(const int32_t* __restrict__ order, int64_t n_grou
   items[q] = r;
 }
 
+inline int log2_pow2(uint64_t v) {  // v a power of two
+  int b = 0;
+  while ((uint64_t(1) << b) < v) ++b;
+  return b;
+}
+
 inline unsigned grid_for(int64_t n, int threads) {
   return unsigned((n + threads - 1) / threads);
 }
@@ -744,14 +744,15 @@ int build_plan_impl(const int32_t* coords, int64_t n, int32_t stride, int64_t ta
     int cur = 0;
     SMC_TRY(radix_sort(sc.ckeys, sc.svals, 0, n, 64, sc.hist, s, &cur));
     k_sorted_dups<<<grid_for(n, 256), 256, 0, s>>>(sc.ckeys[cur], n, plan->status);
-    k_neighbors_sorted<<<grid_for(n, kNbrVoxels), kNbrThreads, 0, s>>>(
+    k_neighbors_sorted<<<grid_for(n, kNbrWarps), kNbrWarps * 32, 0, s>>>(
         c4, n, stride, sc.ckeys[cur], sc.svals[cur], plan->nbr, plan->mask);
   } else {
     if (cudaMemsetAsync(sc.table, 0xFF, cap * sizeof(Slot), s) != cudaSuccess)
       return SMC_ERR_CUDA;
-    k_insert<<<grid_for(n, 256), 256, 0, s>>>(c4, n, sc.table, cap - 1, plan->status);
-    k_neighbors<<<grid_for(n, kNbrVoxels), kNbrThreads, 0, s>>>(c4, n, stride, sc.table, cap - 1,
-                                                                 plan->nbr, plan->mask);
+    const int shift = 64 - log2_pow2(cap);
+    k_insert<<<grid_for(n, 256), 256, 0, s>>>(c4, n, sc.table, cap - 1, shift, plan->status);
+    k_neighbors<<<grid_for(n, kNbrWarps), kNbrWarps * 32, 0, s>>>(c4, n, stride, sc.table, cap - 1,
+                                                                  shift, plan->nbr, plan->mask);
   }
   SMC_LAUNCHED();
 
@@ -987,9 +988,10 @@ extern "C" int smc_build_neighbor_map_static(const int32_t* coords_dev, int64_t 
       cudaMemsetAsync(&sc->status, 0, sizeof(int32_t), s) != cudaSuccess)
     return SMC_ERR_CUDA;
   const int4* c4 = reinterpret_cast<const int4*>(coords_dev);
-  k_insert<<<grid_for(n, 256), 256, 0, s>>>(c4, n, sc->table, cap - 1, &sc->status);
-  k_neighbors<<<grid_for(n, kNbrVoxels), kNbrThreads, 0, s>>>(c4, n, stride, sc->table, cap - 1,
-                                                               map_dev, sc->mask);
+  const int shift = 64 - log2_pow2(cap);
+  k_insert<<<grid_for(n, 256), 256, 0, s>>>(c4, n, sc->table, cap - 1, shift, &sc->status);
+  k_neighbors<<<grid_for(n, kNbrWarps), kNbrWarps * 32, 0, s>>>(c4, n, stride, sc->table, cap - 1,
+                                                                shift, map_dev, sc->mask);
   if (cudaGetLastError() != cudaSuccess) return SMC_ERR_CUDA;
   int32_t dev_status = 0;
   if (cudaMemcpyAsync(&dev_status, &sc->status, sizeof(int32_t), cudaMemcpyDeviceToHost, s) !=
