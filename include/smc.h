@@ -169,9 +169,9 @@ int smc_build_neighbor_map_static(const int32_t* coords_dev, int64_t n, int32_t 
  *         rounded to nearest; SMC_F32 -- CUDA cores, fp64 accumulation,
  *         output rounded once to fp32.
  * stream: the call is asynchronous on this stream and never synchronises.
- *         Forward calls that use the same handle must be ordered (one stream,
- *         or events): the tensor-core kernel keeps its work counter in the
- *         handle.
+ *         A forward only reads the handle (apart from setting its status
+ *         word on a device error), so forwards on one handle may run on
+ *         different streams at once.
  *
  * Tensor-core path when cin % 64 == 0 and cout % 64 == 0 (f16/bf16); any
  * other cin, cout >= 1 runs on the CUDA-core kernel.  feats and out must not
@@ -202,8 +202,8 @@ int smc_forward(smc_handle_t h, const void* feats, const void* W, void* out, int
  * K, cin, cout, dtype, stream: as for smc_forward (cin and cout are the
  *         forward layer's).  Asynchronous; calls on one handle must be
  *         stream-ordered.  The transposed weights live in a workspace the
- *         handle owns, allocated stream-ordered (cudaMallocAsync) the first
- *         time a call needs more than it holds.
+ *         handle owns, allocated stream-ordered from the library's memory pool
+ *         the first time a call needs more than it holds.
  * Errors: as smc_forward, plus SMC_ERR_OOM.
  */
 int smc_backward_input(smc_handle_t h, const void* grad_out, const void* W, void* grad_in, int K,
@@ -246,7 +246,7 @@ int smc_backward_weight(smc_handle_t h, const void* feats, const void* grad_out,
  * out_n          : host pointer, receives the number of parents m; rows
  *                  [0, m) of both outputs are written.
  * Queued on stream, which the call synchronises to read m back; its scratch
- * is allocated and freed stream-ordered (cudaMallocAsync).
+ * is allocated and freed stream-ordered from the library's memory pool.
  * Errors: SMC_ERR_INVALID, _RANGE (coordinates outside the packing limits;
  * outputs undefined), _OOM, _CUDA, _UNSUPPORTED (n >= 2^31).
  */

@@ -625,10 +625,8 @@ struct Carve {
 // Device counters written by the build and read back once at its end.
 struct BuildCounters {
   int32_t status;
-  uint32_t work_counter[63];   // the tensor-core kernel's item counter (+ finished CTAs)
-  unsigned long long stats[2];  // useful pairs, issued rows x taps
   int32_t total_slots;          // copy of tile_off[n_tiles], for the one read-back
-  int32_t pad;
+  unsigned long long stats[2];  // useful pairs, issued rows x taps
 };
 
 // The plan's arrays in one arena (sizes are upper bounds where they depend on
@@ -722,7 +720,6 @@ int build_plan_impl(const int32_t* coords, int64_t n, int32_t stride, int64_t ta
   pc = Carve{static_cast<uint8_t*>(plan->arena), 0};
   carve_plan(pc, plan, &ctr);
   plan->status = &ctr->status;
-  plan->work_counter = ctr->work_counter;
   if (cudaMemsetAsync(ctr, 0, sizeof(BuildCounters), s) != cudaSuccess) return SMC_ERR_CUDA;
   if (n == 0) return SMC_OK;
 

@@ -39,7 +39,6 @@ struct Plan {
                                   // (room for 27 slots per tile)
   int32_t* out_row = nullptr;     // [n_tiles * 128] voxel written per plan row, -1 = none
   int32_t* status = nullptr;      // device status word
-  uint32_t* work_counter = nullptr;  // tensor-core kernel's item counter (+ finished CTAs)
   // items[G - 1][q]: the q-th work item of G consecutive tiles (G = 1, 2),
   // most taps first, so the largest items are handed out first:
   // {first tile, its tap mask, the next tile's mask (0 if none or G = 1),
