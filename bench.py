@@ -49,7 +49,6 @@ DTYPE_NAME = {"f16": "f16", "bf16": "bf16", "f32": "f32"}
 NCU_TRAFFIC: dict = {
     ("uniform128", 0, "greedy"): 64478208 + 15020544,
     ("resblock64", 0, "greedy"): 97104384 + 30331136,
-    ("uniform64", 0, "greedy"): 4840192 + 0,
 }
 # fp32 features run on the CUDA cores with fp64 accumulation: the ALU bound is
 # the fp64 FMA rate, 148 SMs x 64 fp64 lanes x 2 FLOP x 1.965 GHz.

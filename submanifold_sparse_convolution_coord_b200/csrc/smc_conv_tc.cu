@@ -233,19 +233,49 @@ __device__ __forceinline__ int next_tap(uint32_t& rotated, int r) {
   const int t = b + r;
   return t >= kTaps ? t - kTaps : t;
 }
-template <int G>
-__device__ __forceinline__ uint32_t live_tiles(const Item<G>& it, int tap) {
+// The taps of one stage: ta, and with tap pairing (64-channel inputs, two
+// taps per 128-channel unit) the next tap of the item's list, or -1.
+struct StageTaps {
+  int ta, tb;
+};
+template <bool PAIR>
+__device__ __forceinline__ StageTaps next_stage_taps(uint32_t& rem, int rot) {
+  StageTaps t;
+  t.ta = next_tap(rem, rot);
+  t.tb = (PAIR && rem) ? next_tap(rem, rot) : -1;
+  return t;
+}
+// Sub-chunks of a stage that tile k multiplies (bit s = sub-chunk s): with
+// pairing, sub-chunk s is tap s of the pair; otherwise the KS sub-chunks are
+// consecutive 64-channel chunks of one tap.
+template <int G, int KS, bool PAIR>
+__device__ __forceinline__ uint32_t sub_live(const Item<G>& it, int k, StageTaps t) {
+  const uint32_t m = it.mask[k];
+  if constexpr (PAIR)
+    return ((m >> t.ta) & 1u) | (t.tb >= 0 ? ((m >> t.tb) & 1u) << 1 : 0u);
+  else
+    return ((m >> t.ta) & 1u) ? ((1u << KS) - 1u) : 0u;
+}
+// Tiles of the group with any sub-chunk in the stage (bit k = tile k).
+template <int G, int KS, bool PAIR>
+__device__ __forceinline__ uint32_t stage_live(const Item<G>& it, StageTaps t) {
   uint32_t live = 0;
 #pragma unroll
-  for (int k = 0; k < G; ++k) live |= ((it.mask[k] >> tap) & 1u) << k;
+  for (int k = 0; k < G; ++k) live |= (sub_live<G, KS, PAIR>(it, k, t) != 0u ? 1u : 0u) << k;
   return live;
+}
+// Gather-index slot of tile k's tap t (the tile has the tap).
+template <int G>
+__device__ __forceinline__ int index_slot(const Item<G>& it, int k, int t) {
+  return it.slot0[k] + __popc(it.mask[k] & ((1u << t) - 1u));
 }
 
 // NA: A units in flight (16 KS KB each), NW: W slices in flight, NQ gather
 // groups of WPS warps, NBUF accumulator sets in tensor memory (2: the epilogue
 // of one item overlaps the MMAs of the next; 1: room for two 256-column
-// tiles), KS: 64-channel sub-chunks per unit.
-template <int BN, int NA, int NW, int G, int WPS, int NQ, bool BF16, int NBUF, int KS>
+// tiles), KS: 64-channel sub-chunks per unit, PAIR: the two sub-chunks are
+// two taps of 64-channel rows (else KS chunks of one tap).
+template <int BN, int NA, int NW, int G, int WPS, int NQ, bool BF16, int NBUF, int KS, bool PAIR>
 __global__ void __launch_bounds__(threads_for(NQ, WPS), 1)
 k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap fmap,
           const ConvArgs args) {
@@ -262,6 +292,8 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
   static_assert(NW * G <= NA, "MMA warps drift by at most one A slot phase");
   static_assert(NBUF == 1 || NBUF == 2, "accumulator sets");
   static_assert(KS == 1 || KS == 2, "64-channel sub-chunks per unit");
+  static_assert(!PAIR || KS == 2, "tap pairing puts two taps in one 128-channel unit");
+  constexpr int kIdxSlot = (PAIR ? 2 : 1) * kIdxBytes;  // index blocks of one unit
   constexpr int kAUnitBytes = KS * kSubBytes;    // one A unit: 128 rows x 64 KS channels
   constexpr int kWBytes = BN * kBK * 2;          // one W sub-slice: 64 input channels x BN
   constexpr int kWStage = KS * kWBytes;          // the W of one unit
@@ -285,8 +317,8 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
   }
   uint8_t* a_ring = smem_raw;                               // NA x kAUnitBytes
   uint8_t* w_ring = a_ring + NA * kAUnitBytes;              // NW x kWStage
-  int32_t* idx_ring = reinterpret_cast<int32_t*>(w_ring + NW * kWStage);  // NA x 128
-  uint64_t* bars = reinterpret_cast<uint64_t*>(idx_ring + NA * kTileRows);
+  int32_t* idx_ring = reinterpret_cast<int32_t*>(w_ring + NW * kWStage);  // NA x kIdxSlot
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(idx_ring) + NA * kIdxSlot);
   // barriers: afull[NA] aempty[NA] ifull[NA] iempty[NA] wfull[NW] wempty[NW]
   //           tfull[2] tempty[2] info[2] drain[2]
   constexpr int kBars = 4 * NA + 2 * NW + 6 + 2;
@@ -295,7 +327,7 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kb_per_tap = args.cin / (kBK * KS);  // units per tap
+  const int kb_per_tap = PAIR ? 1 : args.cin / (kBK * KS);  // stages per tap (pair)
   const int total_work = args.n_groups * args.n_blocks;
   const uint32_t afull0 = smem_addr(bars);
   const uint32_t aempty0 = afull0 + 8 * NA;
@@ -369,7 +401,8 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
         if (it.w < 0) break;
         uint32_t rem = rotate_taps(it.all, it.rot);
         while (rem && ok) {
-          const int tap = next_tap(rem, it.rot);
+          const StageTaps st = next_stage_taps<PAIR>(rem, it.rot);
+          const int nsub = (PAIR && st.tb < 0) ? 1 : KS;  // an unpaired last tap
           for (int kb = 0; kb < kb_per_tap; ++kb, ++s) {
             const uint32_t ws = s % NW;
             if (!wt.wait(wempty0 + 8 * ws, ((s / NW) & 1) ^ 1)) {
@@ -377,14 +410,18 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
               break;
             }
             const uint32_t full = wfull0 + 8 * ws;
-            mbar_arrive_expect_tx(full, kWStage);
+            mbar_arrive_expect_tx(full, nsub * kWBytes);
             const uint32_t dst = w_base + ws * kWStage;
 #pragma unroll
-            for (int sub = 0; sub < KS; ++sub)
+            for (int sub = 0; sub < KS; ++sub) {
+              if (sub >= nsub) break;
+              const int row = PAIR ? (sub ? st.tb : st.ta) * args.cin
+                                   : st.ta * args.cin + (kb * KS + sub) * kBK;
 #pragma unroll
               for (int jj = 0; jj < BN / 64; ++jj)
-                tma_load_2d(dst + sub * kWBytes + jj * (kBK * 128), &wmap, it.n0 + 64 * jj,
-                            tap * args.cin + (kb * KS + sub) * kBK, full);
+                tma_load_2d(dst + sub * kWBytes + jj * (kBK * 128), &wmap, it.n0 + 64 * jj, row,
+                            full);
+            }
           }
         }
       }
@@ -407,12 +444,12 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
         if (args.dense) continue;  // K = 1 has no gather index
         uint32_t rem = rotate_taps(it.all, it.rot);
         while (rem && ok) {
-          const int tap = next_tap(rem, it.rot);
-          const uint32_t live = live_tiles(it, tap);
+          const StageTaps st = next_stage_taps<PAIR>(rem, it.rot);
           for (int kb = 0; kb < kb_per_tap && ok; ++kb) {
 #pragma unroll
             for (int k = 0; k < G; ++k) {
-              if (!((live >> k) & 1u)) continue;
+              const uint32_t sl = sub_live<G, KS, PAIR>(it, k, st);
+              if (sl == 0u) continue;
               const uint32_t is = u % NA;
               if (!wt.wait(iempty0 + 8 * is, ((u / NA) & 1) ^ 1)) {
                 ok = false;
@@ -421,10 +458,21 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
               // the gathers' reads of this block (generic proxy) come before the
               // bulk copy that overwrites it (async proxy)
               fence_proxy_async_smem();
-              const int slot = it.slot0[k] + __popc(it.mask[k] & ((1u << tap) - 1u));
-              mbar_arrive_expect_tx(ifull0 + 8 * is, kIdxBytes);
-              bulk_load(i_base + is * kIdxBytes, args.gidx + int64_t(slot) * kTileRows, kIdxBytes,
-                        ifull0 + 8 * is);
+              const uint32_t full = ifull0 + 8 * is;
+              if constexpr (PAIR) {
+                mbar_arrive_expect_tx(full, uint32_t(__popc(sl)) * kIdxBytes);
+#pragma unroll
+                for (int sub = 0; sub < 2; ++sub)
+                  if ((sl >> sub) & 1u)
+                    bulk_load(i_base + is * kIdxSlot + sub * kIdxBytes,
+                              args.gidx + int64_t(index_slot(it, k, sub ? st.tb : st.ta)) * kTileRows,
+                              kIdxBytes, full);
+              } else {
+                mbar_arrive_expect_tx(full, kIdxBytes);
+                bulk_load(i_base + is * kIdxSlot,
+                          args.gidx + int64_t(index_slot(it, k, st.ta)) * kTileRows, kIdxBytes,
+                          full);
+              }
               ++u;
             }
           }
@@ -453,12 +501,12 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
       if (it.w < 0) break;
       uint32_t rem = rotate_taps(it.all, it.rot);
       while (rem && ok) {
-        const int tap = next_tap(rem, it.rot);
-        const uint32_t live = live_tiles(it, tap);
+        const StageTaps st = next_stage_taps<PAIR>(rem, it.rot);
         for (int kb = 0; kb < kb_per_tap && ok; ++kb) {
 #pragma unroll
           for (int k = 0; k < G; ++k) {
-            if (!((live >> k) & 1u)) continue;
+            const uint32_t sl = sub_live<G, KS, PAIR>(it, k, st);
+            if (sl == 0u) continue;
             const uint32_t my = u++;
             if (int(my % NQ) != grp) continue;
             const uint32_t slot = my % NA, ph = (my / NA) & 1;
@@ -486,10 +534,13 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
               ok = false;
               break;
             }
-            int v[kInstr];
-            const int32_t* idx = idx_ring + slot * kTileRows + row0 + rsub;
+            constexpr int kSets = PAIR ? 2 : 1;  // index blocks of the unit
+            int v[kSets][kInstr];
+            const int32_t* idx = idx_ring + slot * (kIdxSlot / 4) + row0 + rsub;
 #pragma unroll
-            for (int i = 0; i < kInstr; ++i) v[i] = idx[4 * i];
+            for (int q = 0; q < kSets; ++q)
+#pragma unroll
+              for (int i = 0; i < kInstr; ++i) v[q][i] = idx[q * kTileRows + 4 * i];
             // the block is refilled by a bulk copy (async proxy) once released:
             // order these generic-proxy reads before that write
             fence_proxy_async_smem();
@@ -500,17 +551,20 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
               ok = false;
               break;
             }
-            const uint16_t* src_col = args.feats + kb * (KS * kBK) + chunk * 8;
+            const uint16_t* src_col = args.feats + (PAIR ? 0 : kb * (KS * kBK)) + chunk * 8;
 #pragma unroll
             for (int i = 0; i < kInstr; ++i) {
               const int row = row0 + 4 * i + rsub;
-              const uint16_t* src = v[i] >= 0 ? src_col + int64_t(v[i]) * args.cin : args.feats;
               // 128-byte swizzle: chunk c of row r sits at chunk c ^ (r & 7)
               const uint32_t d = dst + row * 128 + ((chunk ^ (row & 7)) << 4);
 #pragma unroll
-              for (int sub = 0; sub < KS; ++sub)
-                cp_async_16(d + sub * kSubBytes, v[i] >= 0 ? src + sub * kBK : src,
-                            v[i] >= 0 ? 16u : 0u);
+              for (int sub = 0; sub < KS; ++sub) {
+                if (PAIR && !((sl >> sub) & 1u)) continue;  // that tap is not the tile's
+                const int r = v[PAIR ? sub : 0][i];
+                const uint16_t* src =
+                    r >= 0 ? src_col + int64_t(r) * args.cin + (PAIR ? 0 : sub * kBK) : args.feats;
+                cp_async_16(d + sub * kSubBytes, src, r >= 0 ? 16u : 0u);
+              }
             }
             // one arrival per lane on the slot's barrier, made by the hardware
             // once this lane's copies have landed; the MMA warp orders them
@@ -558,8 +612,8 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
       uint32_t started = 0;  // bit k: tile k's accumulator holds a partial sum
       uint32_t rem = rotate_taps(it.all, it.rot);
       while (rem && ok) {
-        const int tap = next_tap(rem, it.rot);
-        const uint32_t live = live_tiles(it, tap);
+        const StageTaps st = next_stage_taps<PAIR>(rem, it.rot);
+        const uint32_t live = stage_live<G, KS, PAIR>(it, st);
         for (int kb = 0; kb < kb_per_tap; ++kb, ++s) {
           const uint32_t ws = s % NW;
           // Both warps wait for every W slice, even one they do not multiply:
@@ -574,7 +628,8 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
           const uint64_t bd = bdesc0 + uint64_t(ws) * (kWStage >> 4);
 #pragma unroll
           for (int k = 0; k < G; ++k) {
-            if (!((live >> k) & 1u)) continue;
+            const uint32_t sl = sub_live<G, KS, PAIR>(it, k, st);
+            if (sl == 0u) continue;
             const uint32_t my = u++;
             if ((uint32_t(k) & 1u) != mine) continue;
             const uint32_t slot = my % NA;
@@ -591,13 +646,16 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
             // never carries, so byte offsets add to the 64-bit value
             const uint64_t ad = adesc0 + uint64_t(slot) * (kAUnitBytes >> 4);
             const uint32_t d_tmem = tmem + (a * G + k) * BN;
-            const uint32_t acc = (started >> k) & 1u;
+            uint32_t acc = (started >> k) & 1u;  // 0 for the tile's first MMA of the item
 #pragma unroll
-            for (int kk = 0; kk < KS * (kBK / 16); ++kk) {
-              const int sub = kk / (kBK / 16), k16 = kk % (kBK / 16);
-              umma_f16(d_tmem, ad + uint64_t(sub) * (kSubBytes >> 4) + 2 * k16,
-                       bd + uint64_t(sub) * (kWBytes >> 4) + (2048 >> 4) * k16, kIdesc,
-                       kk != 0 ? 1u : acc);
+            for (int sub = 0; sub < KS; ++sub) {
+              if (PAIR && !((sl >> sub) & 1u)) continue;  // that tap is not the tile's
+#pragma unroll
+              for (int k16 = 0; k16 < kBK / 16; ++k16) {
+                umma_f16(d_tmem, ad + uint64_t(sub) * (kSubBytes >> 4) + 2 * k16,
+                         bd + uint64_t(sub) * (kWBytes >> 4) + (2048 >> 4) * k16, kIdesc, acc);
+                acc = 1u;
+              }
             }
             umma_commit(aempty0 + 8 * slot);
           }
@@ -729,16 +787,18 @@ bool encode_2d(CUtensorMap* map, bool bf16, const void* base, uint64_t cols, uin
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, int NA, int NW, int G, int WPS, int NQ, bool BF16, int NBUF, int KS>
+template <int BN, int NA, int NW, int G, int WPS, int NQ, bool BF16, int NBUF, int KS,
+          bool PAIR = false>
 int launch_cfg(const Plan& plan, bool dense, const void* feats, const void* W, void* out, int cin,
                int cout, const Epilogue& ep, cudaStream_t stream) {
   constexpr int kWBytes = BN * kBK * 2;
   constexpr int kBars = 4 * NA + 2 * NW + 6 + 2;
   constexpr int kTail = kBars * 8 + 2 * int(sizeof(Item<G>)) + 16;
-  constexpr int kSmem = NA * (KS * kSubBytes + kIdxBytes) + NW * KS * kWBytes + kTail;
+  constexpr int kSmem =
+      NA * (KS * kSubBytes + (PAIR ? 2 : 1) * kIdxBytes) + NW * KS * kWBytes + kTail;
   static_assert(kSmem <= 227 * 1024, "shared memory");
   static_assert(threads_for(NQ, WPS) <= 1024, "threads");
-  auto kern = k_conv_tc<BN, NA, NW, G, WPS, NQ, BF16, NBUF, KS>;
+  auto kern = k_conv_tc<BN, NA, NW, G, WPS, NQ, BF16, NBUF, KS, PAIR>;
   // the shared-memory limit is a per-device function attribute: set it once
   // on each device this configuration runs on
   constexpr int kMaxDev = 64;
@@ -822,12 +882,21 @@ int launch_dtype(const Plan& plan, bool dense, const void* feats, const void* W,
       return launch_cfg<128, 4, 2, 2, 4, 2, BF16, 2, 2>(plan, dense, feats, W, out, cin, cout,
           ep, stream);
     }
+    // 64 input channels and few tiles per SM (a short chain of units per
+    // SM, bound by hand-off latency): two taps per 128-channel unit.  With
+    // many tiles the 64-channel units keep more rows in flight and win.
+    if (cin == 64 && !dense && g1)
+      return launch_cfg<128, 4, 2, 1, 4, 2, BF16, 2, 2, true>(plan, dense, feats, W, out, cin,
+          cout, ep, stream);
     if (g1)
       return launch_cfg<128, 10, 3, 1, 2, 5, BF16, 2, 1>(plan, dense, feats, W, out, cin, cout,
           ep, stream);
     return launch_cfg<128, 10, 3, 2, 2, 5, BF16, 2, 1>(plan, dense, feats, W, out, cin, cout,
         ep, stream);
   }
+  if (cin == 64 && !dense && g1)
+    return launch_cfg<64, 5, 2, 1, 2, 5, BF16, 2, 2, true>(plan, dense, feats, W, out, cin, cout,
+        ep, stream);
   if (g1) return launch_cfg<64, 12, 3, 1, 2, 6, BF16, 2, 1>(plan, dense, feats, W, out, cin, cout,
           ep, stream);
   return launch_cfg<64, 12, 3, 2, 2, 6, BF16, 2, 1>(plan, dense, feats, W, out, cin, cout,
