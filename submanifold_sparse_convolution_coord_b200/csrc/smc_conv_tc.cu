@@ -869,6 +869,10 @@ int launch_dtype(const Plan& plan, bool dense, const void* feats, const void* W,
         (group_override() == 0 && !dense && items2 >= 2 * int64_t(sm_count())))
       return launch_cfg<256, 9, 2, 2, 4, 3, BF16, 1, 1>(plan, dense, feats, W, out, cin, cout,
           ep, stream);
+    // K = 1: 128-channel units (half the hand-offs per multiply)
+    if (dense && cin % 128 == 0)
+      return launch_cfg<256, 3, 2, 1, 4, 3, BF16, 2, 2>(plan, dense, feats, W, out, cin, cout,
+          ep, stream);
     return launch_cfg<256, 9, 2, 1, 4, 3, BF16, 2, 1>(plan, dense, feats, W, out, cin, cout,
         ep, stream);
   }
