@@ -335,6 +335,12 @@ def run_ours(args) -> None:
     flops = useful_flops(pairs, cin, cout)
 
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    # launch-configuration search on this layer (kept in the handle), before
+    # any timed work; --no-autotune keeps the library's fixed rule
+    launch_config = "default rule"
+    if not args.no_autotune:
+        launch_config = binding.conv_config_name(
+            binding.smc_autotune(idx.handle, feats, W, out, K, cin, cout))
 
     def step():
         binding.smc_forward(idx.handle, feats, W, out, K, cin, cout)
@@ -414,6 +420,7 @@ def run_ours(args) -> None:
         "config": {"workload": args.workload, "grid": w.grid, "batch": w.batch,
                    "n_voxels": inp.n, "layer": args.layer, "cin": cin, "cout": cout, "K": K,
                    "occupancy": OCCUPANCY[w.sparsity], "seed": 0, "plan_order": args.order,
+                   "launch_config": launch_config,
                    "l2": "flushed between steps (256 MB write, outside the timed events)",
                    "parallelism": f"replicas x{world}"},
         "conv_ms": conv_ms_max,
@@ -468,6 +475,8 @@ def main(argv=None) -> None:
                     help="layer of the workload to time (resblock64: 0 = 3x3x3 512->512, "
                          "1 = 1x1x1 512->1024)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-autotune", action="store_true",
+                    help="use the fixed launch-configuration rule instead of the search")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     args = ap.parse_args(argv)
     if args.warmup < 3:

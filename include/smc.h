@@ -185,6 +185,28 @@ int smc_forward(smc_handle_t h, const void* feats, const void* W, void* out, int
                 int cin, int cout, int dtype, smc_stream_t stream);
 
 /*
+ * Launch-configuration search for smc_forward ("Metal-native replacement for
+ * flex_gemm bottleneck?", "Open": autotuning of the tile shape and schedule).
+ * Runs every tensor-core launch configuration valid for this layer shape
+ * (output-column block, tiles per work item, 128-channel units or tap pairs)
+ * on the given buffers, once to warm up and three times timed with CUDA
+ * events on `stream`, and keeps the fastest in the handle for this
+ * (K, cin, cout, dtype): later smc_forward / smc_forward_ex calls of that
+ * shape use it.  Without a search they use a fixed rule.
+ * Arguments as smc_forward; out is overwritten (it holds the forward result
+ * afterwards).  chosen (host pointer, may be null) receives the configuration
+ * id (name: smc_conv_config_name), or -1 when the shape runs on the CUDA
+ * cores (nothing to choose).  Synchronises the stream.
+ * Errors: as smc_forward; SMC_ERR_TIMEOUT when a candidate's device-side wait
+ * gave up (the handle then keeps its previous choice).
+ */
+int smc_autotune(smc_handle_t h, const void* feats, const void* W, void* out, int K, int cin,
+                 int cout, int dtype, smc_stream_t stream, int* chosen);
+
+/* Static name of a launch configuration id ("cuda-cores" for -1). */
+const char* smc_conv_config_name(int config);
+
+/*
  * Input gradient of smc_forward ("Metal-native replacement for flex_gemm
  * bottleneck?", "Fixed" / "Open": the bwd-input pass next to fwd):
  *

@@ -33,7 +33,7 @@ EXPORTS = (
     "smc_get_plan_stats", "smc_get_sizes", "smc_get_tile_plan", "smc_device_status",
     "smc_destroy", "smc_status_string", "smc_version", "smc_build_neighbor_map_static",
     "smc_backward_input", "smc_backward_weight", "smc_downsample2", "smc_subdivide2",
-    "smc_forward_ex",
+    "smc_forward_ex", "smc_autotune", "smc_conv_config_name",
 )
 
 
@@ -89,9 +89,12 @@ def lib() -> ctypes.CDLL:
     L.smc_status_string.restype = ctypes.c_char_p
     L.smc_version.argtypes = []
     L.smc_build_neighbor_map_static.argtypes = [p, i64, i32, p, p]
+    L.smc_autotune.argtypes = [p, p, p, p, i, i, i, i, p, ctypes.POINTER(i)]
+    L.smc_conv_config_name.argtypes = [i]
+    L.smc_conv_config_name.restype = ctypes.c_char_p
     for name in EXPORTS:
         fn = getattr(L, name)
-        if name not in ("smc_destroy", "smc_status_string"):
+        if name not in ("smc_destroy", "smc_status_string", "smc_conv_config_name"):
             fn.restype = ctypes.c_int
     _lib = L
     return L
@@ -156,6 +159,33 @@ def smc_forward(handle: int, feats: torch.Tensor, W: torch.Tensor, out: torch.Te
                                ctypes.c_void_p(op), int(K), int(cin), int(cout),
                                DTYPE_CODE[dtype], _stream(stream, feats.device))
     _check(rc, "smc_forward")
+
+
+def smc_autotune(handle: int, feats: torch.Tensor, W: torch.Tensor, out: torch.Tensor, K: int,
+                 cin: int, cout: int, stream: Optional[torch.cuda.Stream] = None) -> int:
+    """Time the valid launch configurations on these buffers and keep the
+    fastest in the handle; returns its id (-1: CUDA cores).  out is
+    overwritten with the forward result."""
+    dtype = feats.dtype
+    if dtype not in DTYPE_CODE:
+        raise ValueError(f"unsupported dtype {dtype}")
+    fp = _dev_ptr(feats, "feats", dtype)
+    wp = _dev_ptr(W, "W", dtype)
+    op = _dev_ptr(out, "out", dtype)
+    if W.device != feats.device or out.device != feats.device:
+        raise ValueError("feats, W and out must be on one device")
+    chosen = ctypes.c_int(-1)
+    with torch.cuda.device(feats.device):
+        rc = lib().smc_autotune(ctypes.c_void_p(handle), ctypes.c_void_p(fp), ctypes.c_void_p(wp),
+                                ctypes.c_void_p(op), int(K), int(cin), int(cout),
+                                DTYPE_CODE[dtype], _stream(stream, feats.device),
+                                ctypes.byref(chosen))
+    _check(rc, "smc_autotune")
+    return chosen.value
+
+
+def conv_config_name(config: int) -> str:
+    return lib().smc_conv_config_name(int(config)).decode()
 
 
 def smc_forward_ex(handle: int, feats: torch.Tensor, W: torch.Tensor, out: torch.Tensor, K: int,
@@ -343,6 +373,15 @@ class SubMIndex:
 
     def status(self) -> int:
         return smc_device_status(self.handle, self.device)
+
+    def autotune(self, feats: torch.Tensor, W: torch.Tensor, K: int = 3) -> str:
+        """Choose the fastest launch configuration for this layer shape on
+        these inputs (kept for later forwards of the shape); returns its name."""
+        taps, cin, cout = W.shape
+        if taps != K ** 3 or cin != feats.shape[1] or feats.shape[0] != self.n:
+            raise ValueError("feats must be [N, Cin] and W [K^3, Cin, Cout]")
+        out = torch.empty((self.n, cout), dtype=feats.dtype, device=feats.device)
+        return conv_config_name(smc_autotune(self.handle, feats, W, out, K, cin, cout))
 
     def forward(self, feats: torch.Tensor, W: torch.Tensor, K: int = 3,
                 out: Optional[torch.Tensor] = None, bias: Optional[torch.Tensor] = None,

@@ -14,6 +14,29 @@ struct smc_index {
   // grown stream-ordered; calls on one handle are stream-ordered
   void* work = nullptr;
   size_t work_bytes = 0;
+  // launch configurations chosen by smc_autotune, per layer shape
+  struct Tuned {
+    int K, cin, cout, dtype, cfg;
+  };
+  static constexpr int kMaxTuned = 16;
+  Tuned tuned[kMaxTuned];
+  int n_tuned = 0;
+  int tuned_config(int K, int cin, int cout, int dtype) const {
+    for (int i = 0; i < n_tuned; ++i)
+      if (tuned[i].K == K && tuned[i].cin == cin && tuned[i].cout == cout &&
+          tuned[i].dtype == dtype)
+        return tuned[i].cfg;
+    return -1;
+  }
+  void set_tuned(int K, int cin, int cout, int dtype, int cfg) {
+    for (int i = 0; i < n_tuned; ++i)
+      if (tuned[i].K == K && tuned[i].cin == cin && tuned[i].cout == cout &&
+          tuned[i].dtype == dtype) {
+        tuned[i].cfg = cfg;
+        return;
+      }
+    if (n_tuned < kMaxTuned) tuned[n_tuned++] = Tuned{K, cin, cout, dtype, cfg};
+  }
 };
 
 namespace {
@@ -62,9 +85,9 @@ int check_call(smc_index* h, int K, int cin, int cout, int dtype) {
 }
 
 int conv(const smc::Plan& plan, bool dense, const void* x, const void* W, void* y, int cin,
-         int cout, int dtype, const smc::Epilogue& ep, cudaStream_t s) {
+         int cout, int dtype, const smc::Epilogue& ep, cudaStream_t s, int cfg = -1) {
   if (smc::conv_tc_supported(cin, cout, dtype))
-    return smc::launch_conv_tc(plan, dense, x, W, y, cin, cout, dtype, ep, s);
+    return smc::launch_conv_tc(plan, dense, x, W, y, cin, cout, dtype, ep, s, cfg);
   return smc::launch_conv_simt(plan, dense, x, W, y, cin, cout, dtype, ep, s);
 }
 
@@ -160,12 +183,70 @@ int smc_forward_ex(smc_handle_t h, const void* feats, const void* W, void* out, 
   if (!feats || !W || !out) return SMC_ERR_INVALID;
   if (!aligned16(feats) || !aligned16(W) || !aligned16(out)) return SMC_ERR_INVALID;
   return conv(plan, K == 1, feats, W, out, cin, cout, dtype, e,
-              reinterpret_cast<cudaStream_t>(stream));
+              reinterpret_cast<cudaStream_t>(stream), h->tuned_config(K, cin, cout, dtype));
 }
 
 int smc_forward(smc_handle_t h, const void* feats, const void* W, void* out, int K, int cin,
                 int cout, int dtype, smc_stream_t stream) {
   return smc_forward_ex(h, feats, W, out, K, cin, cout, dtype, nullptr, stream);
+}
+
+const char* smc_conv_config_name(int config) { return smc::conv_config_name(config); }
+
+int smc_autotune(smc_handle_t h, const void* feats, const void* W, void* out, int K, int cin,
+                 int cout, int dtype, smc_stream_t stream, int* chosen) {
+  if (chosen) *chosen = -1;
+  const int rc = check_call(h, K, cin, cout, dtype);
+  if (rc != SMC_OK) return rc;
+  const smc::Plan& plan = h->plan;
+  if (plan.n == 0 || !smc::conv_tc_supported(cin, cout, dtype)) return SMC_OK;
+  if (!feats || !W || !out) return SMC_ERR_INVALID;
+  if (!aligned16(feats) || !aligned16(W) || !aligned16(out)) return SMC_ERR_INVALID;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool dense = K == 1;
+  cudaEvent_t ev[2];
+  if (cudaEventCreate(&ev[0]) != cudaSuccess) return SMC_ERR_CUDA;
+  if (cudaEventCreate(&ev[1]) != cudaSuccess) {
+    cudaEventDestroy(ev[0]);
+    return SMC_ERR_CUDA;
+  }
+  int best = -1, status = SMC_OK;
+  float best_ms = 0.f;
+  const smc::Epilogue none;
+  for (int cfg = 0; cfg < smc::kConvConfigs && status == SMC_OK; ++cfg) {
+    if (!smc::conv_config_valid(cfg, dense, cin, cout)) continue;
+    float t = 0.f;
+    for (int rep = 0; rep < 4 && status == SMC_OK; ++rep) {
+      if (cudaEventRecord(ev[0], s) != cudaSuccess) status = SMC_ERR_CUDA;
+      if (status == SMC_OK)
+        status = smc::launch_conv_tc(plan, dense, feats, W, out, cin, cout, dtype, none, s, cfg);
+      if (status == SMC_OK && (cudaEventRecord(ev[1], s) != cudaSuccess ||
+                               cudaEventSynchronize(ev[1]) != cudaSuccess))
+        status = SMC_ERR_CUDA;
+      float ms = 0.f;
+      if (status == SMC_OK && cudaEventElapsedTime(&ms, ev[0], ev[1]) != cudaSuccess)
+        status = SMC_ERR_CUDA;
+      if (rep == 1 || (rep > 1 && ms < t)) t = ms;  // the first run warms up
+    }
+    if (status == SMC_OK && (best < 0 || t < best_ms)) {
+      best = cfg;
+      best_ms = t;
+    }
+  }
+  cudaEventDestroy(ev[0]);
+  cudaEventDestroy(ev[1]);
+  if (status != SMC_OK) return status;
+  // a candidate whose bounded wait gave up leaves the choice as it was
+  status = smc_device_status(h, stream);
+  if (status != SMC_OK) return status;
+  if (best >= 0) {
+    h->set_tuned(K, cin, cout, dtype, best);
+    // leave out holding the chosen configuration's result
+    status = smc::launch_conv_tc(plan, dense, feats, W, out, cin, cout, dtype, none, s, best);
+    if (status != SMC_OK) return status;
+  }
+  if (chosen) *chosen = best;
+  return SMC_OK;
 }
 
 int smc_backward_input(smc_handle_t h, const void* grad_out, const void* W, void* grad_in, int K,

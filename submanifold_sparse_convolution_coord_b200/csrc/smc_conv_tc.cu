@@ -852,14 +852,76 @@ int group_override() {
   return v;
 }
 
+// The launch configurations, by id (see the ConvConfig enumeration in
+// smc_internal.h for what each one is).
 template <bool BF16>
-int launch_dtype(const Plan& plan, bool dense, const void* feats, const void* W, void* out,
-                 int cin, int cout, const Epilogue& ep, cudaStream_t stream) {
+int launch_config(int cfg, const Plan& plan, bool dense, const void* feats, const void* W,
+                  void* out, int cin, int cout, const Epilogue& ep, cudaStream_t stream) {
+#define SMC_CFG(...) return launch_cfg<__VA_ARGS__>(plan, dense, feats, W, out, cin, cout, ep, stream)
+  switch (cfg) {  //            BN  NA NW G WPS NQ        NBUF KS PAIR
+    case kCfg256G2: SMC_CFG(256, 9, 2, 2, 4, 3, BF16, 1, 1);
+    case kCfg256G1: SMC_CFG(256, 9, 2, 1, 4, 3, BF16, 2, 1);
+    case kCfg256G1K2: SMC_CFG(256, 3, 2, 1, 4, 3, BF16, 2, 2);
+    case kCfg128G2K2: SMC_CFG(128, 4, 2, 2, 4, 2, BF16, 2, 2);
+    case kCfg128G1K2: SMC_CFG(128, 4, 2, 1, 4, 2, BF16, 2, 2);
+    case kCfg128G1Pair: SMC_CFG(128, 4, 2, 1, 4, 2, BF16, 2, 2, true);
+    case kCfg128G2: SMC_CFG(128, 10, 3, 2, 2, 5, BF16, 2, 1);
+    case kCfg128G1: SMC_CFG(128, 10, 3, 1, 2, 5, BF16, 2, 1);
+    case kCfg64G1Pair: SMC_CFG(64, 5, 2, 1, 2, 5, BF16, 2, 2, true);
+    case kCfg64G2: SMC_CFG(64, 12, 3, 2, 2, 6, BF16, 2, 1);
+    case kCfg64G1: SMC_CFG(64, 12, 3, 1, 2, 6, BF16, 2, 1);
+    default: return SMC_ERR_INVALID;
+  }
+#undef SMC_CFG
+}
+
+}  // namespace
+
+bool conv_config_valid(int cfg, bool dense, int cin, int cout) {
+  if (cin % 64 != 0 || cout % 64 != 0) return false;
+  switch (cfg) {
+    case kCfg256G2:
+    case kCfg256G1:
+      return cout % 256 == 0;
+    case kCfg256G1K2:
+      return cout % 256 == 0 && cin % 128 == 0;
+    case kCfg128G2K2:
+    case kCfg128G1K2:
+      return cout % 128 == 0 && cin % 128 == 0;
+    case kCfg128G1Pair:
+      return cout % 128 == 0 && cin == 64 && !dense;
+    case kCfg128G2:
+    case kCfg128G1:
+      return cout % 128 == 0;
+    case kCfg64G1Pair:
+      return cin == 64 && !dense;
+    case kCfg64G2:
+    case kCfg64G1:
+      return true;
+    default:
+      return false;
+  }
+}
+
+const char* conv_config_name(int cfg) {
+  static const char* const kNames[kConvConfigs] = {
+      "bn256-g2",     "bn256-g1",  "bn256-g1-k128", "bn128-g2-k128", "bn128-g1-k128",
+      "bn128-g1-pair", "bn128-g2",  "bn128-g1",      "bn64-g1-pair",  "bn64-g2",
+      "bn64-g1"};
+  return cfg >= 0 && cfg < kConvConfigs ? kNames[cfg] : "cuda-cores";
+}
+
+int conv_default_config(const Plan& plan, bool dense, int cin, int cout) {
+  // Test and tuning override, read at every call: SMC_TC_CONFIG=<id> forces
+  // a configuration wherever it is valid.
+  if (const char* e = std::getenv("SMC_TC_CONFIG")) {
+    const int c = std::atoi(e);
+    if (conv_config_valid(c, dense, cin, cout)) return c;
+  }
   // Few tiles per SM: one tile per work item, so every SM gets work and no SM
   // runs two heavy tiles back to back.
   const bool small = plan.n_tiles < int64_t(6) * sm_count();
   const bool g1 = group_override() == 1 || (small && group_override() != 2);
-  //                          BN  NA NW G WPS NQ        NBUF KS
   if (cout % 256 == 0) {
     // sparse: two 256-column tiles per item share each W slice (one
     // accumulator set), as long as that leaves at least two items per SM;
@@ -867,47 +929,24 @@ int launch_dtype(const Plan& plan, bool dense, const void* feats, const void* W,
     const int64_t items2 = (plan.n_tiles + 1) / 2 * (cout / 256);
     if (group_override() == 2 ||
         (group_override() == 0 && !dense && items2 >= 2 * int64_t(sm_count())))
-      return launch_cfg<256, 9, 2, 2, 4, 3, BF16, 1, 1>(plan, dense, feats, W, out, cin, cout,
-          ep, stream);
+      return kCfg256G2;
     // K = 1: 128-channel units (half the hand-offs per multiply)
-    if (dense && cin % 128 == 0)
-      return launch_cfg<256, 3, 2, 1, 4, 3, BF16, 2, 2>(plan, dense, feats, W, out, cin, cout,
-          ep, stream);
-    return launch_cfg<256, 9, 2, 1, 4, 3, BF16, 2, 1>(plan, dense, feats, W, out, cin, cout,
-        ep, stream);
+    if (dense && cin % 128 == 0) return kCfg256G1K2;
+    return kCfg256G1;
   }
   if (cout % 128 == 0) {
     // 128 input channels per unit where Cin allows: half the hand-offs per
     // multiply of the 64-channel unit
-    if (cin % 128 == 0) {
-      if (g1)
-        return launch_cfg<128, 4, 2, 1, 4, 2, BF16, 2, 2>(plan, dense, feats, W, out, cin, cout,
-            ep, stream);
-      return launch_cfg<128, 4, 2, 2, 4, 2, BF16, 2, 2>(plan, dense, feats, W, out, cin, cout,
-          ep, stream);
-    }
+    if (cin % 128 == 0) return g1 ? kCfg128G1K2 : kCfg128G2K2;
     // 64 input channels and few tiles per SM (a short chain of units per
     // SM, bound by hand-off latency): two taps per 128-channel unit.  With
     // many tiles the 64-channel units keep more rows in flight and win.
-    if (cin == 64 && !dense && g1)
-      return launch_cfg<128, 4, 2, 1, 4, 2, BF16, 2, 2, true>(plan, dense, feats, W, out, cin,
-          cout, ep, stream);
-    if (g1)
-      return launch_cfg<128, 10, 3, 1, 2, 5, BF16, 2, 1>(plan, dense, feats, W, out, cin, cout,
-          ep, stream);
-    return launch_cfg<128, 10, 3, 2, 2, 5, BF16, 2, 1>(plan, dense, feats, W, out, cin, cout,
-        ep, stream);
+    if (cin == 64 && !dense && g1) return kCfg128G1Pair;
+    return g1 ? kCfg128G1 : kCfg128G2;
   }
-  if (cin == 64 && !dense && g1)
-    return launch_cfg<64, 5, 2, 1, 2, 5, BF16, 2, 2, true>(plan, dense, feats, W, out, cin, cout,
-        ep, stream);
-  if (g1) return launch_cfg<64, 12, 3, 1, 2, 6, BF16, 2, 1>(plan, dense, feats, W, out, cin, cout,
-          ep, stream);
-  return launch_cfg<64, 12, 3, 2, 2, 6, BF16, 2, 1>(plan, dense, feats, W, out, cin, cout,
-      ep, stream);
+  if (cin == 64 && !dense && g1) return kCfg64G1Pair;
+  return g1 ? kCfg64G1 : kCfg64G2;
 }
-
-}  // namespace
 
 // A test sets SMC_DEBUG_WAIT_LIMIT_NS tiny to exercise the abort path.
 uint64_t wait_limit_ns() {
@@ -925,12 +964,15 @@ bool conv_tc_supported(int cin, int cout, int dtype) {
 }
 
 int launch_conv_tc(const Plan& plan, bool dense, const void* feats, const void* W, void* out,
-                   int cin, int cout, int dtype, const Epilogue& ep, cudaStream_t stream) {
+                   int cin, int cout, int dtype, const Epilogue& ep, cudaStream_t stream,
+                   int cfg) {
   if (plan.n == 0) return SMC_OK;
   if (!conv_tc_supported(cin, cout, dtype)) return SMC_ERR_UNSUPPORTED;
+  if (cfg < 0) cfg = conv_default_config(plan, dense, cin, cout);
+  if (!conv_config_valid(cfg, dense, cin, cout)) return SMC_ERR_INVALID;
   if (dtype == SMC_BF16)
-    return launch_dtype<true>(plan, dense, feats, W, out, cin, cout, ep, stream);
-  return launch_dtype<false>(plan, dense, feats, W, out, cin, cout, ep, stream);
+    return launch_config<true>(cfg, plan, dense, feats, W, out, cin, cout, ep, stream);
+  return launch_config<false>(cfg, plan, dense, feats, W, out, cin, cout, ep, stream);
 }
 
 }  // namespace smc

@@ -76,9 +76,30 @@ void free_plan(Plan* plan);
 
 // Tensor-core convolution (smc_conv_tc.cu).  feats/W/out in f16 or bf16.
 // dense = true runs the K = 1 form (rows in order, one tap, no plan arrays).
+// cfg selects a launch configuration (ConvConfig), -1 the default rule.
 int launch_conv_tc(const Plan& plan, bool dense, const void* feats, const void* W, void* out,
-                   int cin, int cout, int dtype, const Epilogue& ep, cudaStream_t stream);
+                   int cin, int cout, int dtype, const Epilogue& ep, cudaStream_t stream,
+                   int cfg = -1);
 bool conv_tc_supported(int cin, int cout, int dtype);
+// Launch configurations of the tensor-core kernel: output-column block (BN),
+// tiles per work item (G), 128-channel units (k128) or tap pairs (pair).
+enum ConvConfig : int {
+  kCfg256G2 = 0,  // BN 256, two tiles per item sharing each W slice, one accumulator set
+  kCfg256G1,      // BN 256, one tile per item
+  kCfg256G1K2,    // BN 256, one tile per item, 128-channel units
+  kCfg128G2K2,    // BN 128, two tiles per item, 128-channel units
+  kCfg128G1K2,    // BN 128, one tile per item, 128-channel units
+  kCfg128G1Pair,  // BN 128, one tile per item, two taps per unit (Cin = 64, K = 3)
+  kCfg128G2,      // BN 128, two tiles per item, 64-channel units
+  kCfg128G1,      // BN 128, one tile per item, 64-channel units
+  kCfg64G1Pair,   // BN 64, one tile per item, two taps per unit (Cin = 64, K = 3)
+  kCfg64G2,       // BN 64, two tiles per item, 64-channel units
+  kCfg64G1,       // BN 64, one tile per item, 64-channel units
+  kConvConfigs
+};
+bool conv_config_valid(int cfg, bool dense, int cin, int cout);
+int conv_default_config(const Plan& plan, bool dense, int cin, int cout);
+const char* conv_config_name(int cfg);
 
 // Stable LSD radix sort of (key, value) pairs by the low `bits` bits of the
 // key, 8 bits per pass (smc_sort.cu).  Reads buffer `cur`, ping-pongs between

@@ -282,3 +282,48 @@ def test_bounded_wait_abort_path(limit_ns, must_abort):
     ref, scale = oracle_conv(coords, feats, W, 3)
     check_conv(out, ref, scale, "after abort runs")
     idx.close()
+
+
+# (cin, cout, dtype, K): every launch configuration family appears in one of these
+AUTOTUNE_SHAPES = [(128, 128, "f16", 3), (64, 64, "bf16", 3), (64, 128, "f16", 3),
+                   (128, 256, "bf16", 3), (256, 256, "bf16", 1), (64, 256, "f16", 1)]
+
+
+@pytest.mark.parametrize("shape", AUTOTUNE_SHAPES, ids=lambda s: "{}x{}_{}_K{}".format(*s))
+def test_every_launch_configuration(shape, monkeypatch):
+    """Each tensor-core launch configuration valid for the shape (forced
+    through SMC_TC_CONFIG, read at every call) matches the oracle, and the
+    configuration search picks a valid one whose forward matches too."""
+    from submanifold_sparse_convolution_coord_b200 import binding
+    cin, cout, dt, K = shape
+    coords, feats, W = synth.random_case(50 + cin + cout, 3000, 24, 1, cin, cout, K, dt, True)
+    ref, scale = oracle_conv(coords, feats, W, K)
+    c = torch.from_numpy(np.ascontiguousarray(coords, dtype=np.int32)).to(DEV)
+    idx = SubMIndex(c)
+    f, w = feats.to(DEV), W.to(DEV)
+    for cfg in range(11):
+        monkeypatch.setenv("SMC_TC_CONFIG", str(cfg))
+        out = idx.forward(f, w, K=K)
+        torch.cuda.synchronize()
+        assert idx.status() == 0
+        check_conv(out, ref, scale, f"{shape} config {binding.conv_config_name(cfg)}")
+    monkeypatch.delenv("SMC_TC_CONFIG")
+    name = idx.autotune(f, w, K=K)
+    assert name not in ("cuda-cores", "")
+    out = idx.forward(f, w, K=K)
+    torch.cuda.synchronize()
+    assert idx.status() == 0
+    check_conv(out, ref, scale, f"{shape} tuned {name}")
+    idx.close()
+
+
+def test_autotune_cuda_core_shapes():
+    """fp32 (and off-grid channel counts) run on the CUDA cores: nothing to
+    choose, and the forward is unchanged."""
+    coords, feats, W = synth.random_case(61, 800, 12, 1, 16, 16, 3, "f32", True)
+    c = torch.from_numpy(np.ascontiguousarray(coords, dtype=np.int32)).to(DEV)
+    idx = SubMIndex(c)
+    assert idx.autotune(feats.to(DEV), W.to(DEV), K=3) == "cuda-cores"
+    ref, scale = oracle_conv(coords, feats, W, 3)
+    check_conv(idx.forward(feats.to(DEV), W.to(DEV), K=3), ref, scale, "f32 after autotune")
+    idx.close()
