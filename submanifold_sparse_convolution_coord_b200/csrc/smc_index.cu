@@ -18,10 +18,10 @@
 //   5. items    for work items of one and of two consecutive tiles, the
 //               groups in decreasing order of their union's tap count (one
 //               block-wide stable counting sort, or a radix pass for more
-//               than 49,152 tiles), so the convolution hands out its largest
+//               than 49,152 tiles), so the convolution deals its largest
 //               items first, each written as a 16-byte record (first tile,
-//               tap masks, first gather-index slot) the convolution's
-//               scheduler reads with one load.
+//               tap masks, first gather-index slot) that each role of the
+//               convolution reads with one load.
 #include <algorithm>
 #include <cstdio>
 #include <cstring>
