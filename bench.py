@@ -47,8 +47,10 @@ DTYPE_NAME = {"f16": "f16", "bf16": "bf16", "f32": "f32"}
 # launch (bytes; profiles/k_conv_tc_*.md).  Cases not captured with the current
 # kernel report null.
 NCU_TRAFFIC: dict = {
-    ("uniform128", 0, "greedy"): 64478208 + 15020544,
-    ("resblock64", 0, "greedy"): 97104384 + 30331136,
+    ("uniform128", 0, "greedy"): 64355584 + 14522624,
+    ("resblock64", 0, "greedy"): 99606784 + 32485376,
+    ("resblock64", 1, "greedy"): 57634048 + 59953664,
+    ("uniform64", 0, "greedy"): 4848640 + 0,
 }
 # fp32 features run on the CUDA cores with fp64 accumulation: the ALU bound is
 # the fp64 FMA rate, 148 SMs x 64 fp64 lanes x 2 FLOP x 1.965 GHz.
