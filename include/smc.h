@@ -207,6 +207,32 @@ int smc_autotune(smc_handle_t h, const void* feats, const void* W, void* out, in
 const char* smc_conv_config_name(int config);
 
 /*
+ * smc_autotune with the row order of the tile plan searched too
+ * (search_orders != 0, K = 3): for SMC_ORDER_MASK and SMC_ORDER_GREEDY the
+ * handle's plan is rebuilt in that order (smc_replan) and every launch
+ * configuration timed; the handle keeps the fastest (order, configuration).
+ * The order belongs to the whole handle, so it applies to every layer that
+ * uses it.  chosen_order (host pointer, may be null) receives the order.
+ * Synchronises the device; no other call may use the handle meanwhile.
+ * Errors: as smc_autotune, plus those of smc_replan.
+ */
+int smc_autotune_ex(smc_handle_t h, const void* feats, const void* W, void* out, int K, int cin,
+                    int cout, int dtype, int search_orders, smc_stream_t stream,
+                    int* chosen_config, int* chosen_order);
+
+/*
+ * Rebuild the handle's tile plan (row order, tiles, gather index, work items,
+ * tap lists) in another row order (enum smc_order) from the neighbour map
+ * and tap masks it already holds; the neighbour map is unchanged and the
+ * coordinates are not needed.  Waits for all work on the handle's device
+ * first (a forward in flight reads the plan), then runs on `stream` and
+ * synchronises it.  Configurations chosen by smc_autotune are dropped.
+ * Errors: SMC_ERR_INVALID (null handle, bad order, another current device),
+ * SMC_ERR_OOM (scratch), SMC_ERR_CUDA.
+ */
+int smc_replan(smc_handle_t h, int order, smc_stream_t stream);
+
+/*
  * Input gradient of smc_forward ("Metal-native replacement for flex_gemm
  * bottleneck?", "Fixed" / "Open": the bwd-input pass next to fwd):
  *

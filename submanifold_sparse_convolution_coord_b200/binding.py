@@ -33,7 +33,7 @@ EXPORTS = (
     "smc_get_plan_stats", "smc_get_sizes", "smc_get_tile_plan", "smc_device_status",
     "smc_destroy", "smc_status_string", "smc_version", "smc_build_neighbor_map_static",
     "smc_backward_input", "smc_backward_weight", "smc_downsample2", "smc_subdivide2",
-    "smc_forward_ex", "smc_autotune", "smc_conv_config_name",
+    "smc_forward_ex", "smc_autotune", "smc_conv_config_name", "smc_autotune_ex", "smc_replan",
 )
 
 
@@ -90,6 +90,9 @@ def lib() -> ctypes.CDLL:
     L.smc_version.argtypes = []
     L.smc_build_neighbor_map_static.argtypes = [p, i64, i32, p, p]
     L.smc_autotune.argtypes = [p, p, p, p, i, i, i, i, p, ctypes.POINTER(i)]
+    L.smc_autotune_ex.argtypes = [p, p, p, p, i, i, i, i, i, p, ctypes.POINTER(i),
+                                  ctypes.POINTER(i)]
+    L.smc_replan.argtypes = [p, i, p]
     L.smc_conv_config_name.argtypes = [i]
     L.smc_conv_config_name.restype = ctypes.c_char_p
     for name in EXPORTS:
@@ -182,6 +185,38 @@ def smc_autotune(handle: int, feats: torch.Tensor, W: torch.Tensor, out: torch.T
                                 ctypes.byref(chosen))
     _check(rc, "smc_autotune")
     return chosen.value
+
+
+def smc_autotune_ex(handle: int, feats: torch.Tensor, W: torch.Tensor, out: torch.Tensor, K: int,
+                    cin: int, cout: int, search_orders: bool = True,
+                    stream: Optional[torch.cuda.Stream] = None) -> tuple:
+    """smc_autotune, with the plan's row order searched as well; returns
+    (configuration id, order name)."""
+    dtype = feats.dtype
+    if dtype not in DTYPE_CODE:
+        raise ValueError(f"unsupported dtype {dtype}")
+    fp = _dev_ptr(feats, "feats", dtype)
+    wp = _dev_ptr(W, "W", dtype)
+    op = _dev_ptr(out, "out", dtype)
+    if W.device != feats.device or out.device != feats.device:
+        raise ValueError("feats, W and out must be on one device")
+    cfg, order = ctypes.c_int(-1), ctypes.c_int(-1)
+    with torch.cuda.device(feats.device):
+        rc = lib().smc_autotune_ex(ctypes.c_void_p(handle), ctypes.c_void_p(fp),
+                                   ctypes.c_void_p(wp), ctypes.c_void_p(op), int(K), int(cin),
+                                   int(cout), DTYPE_CODE[dtype], int(bool(search_orders)),
+                                   _stream(stream, feats.device), ctypes.byref(cfg),
+                                   ctypes.byref(order))
+    _check(rc, "smc_autotune_ex")
+    names = {v: k for k, v in ORDER_CODE.items()}
+    return cfg.value, names.get(order.value, str(order.value))
+
+
+def smc_replan(handle: int, order: str, device: torch.device,
+               stream: Optional[torch.cuda.Stream] = None) -> None:
+    with torch.cuda.device(device):
+        rc = lib().smc_replan(ctypes.c_void_p(handle), ORDER_CODE[order], _stream(stream, device))
+    _check(rc, "smc_replan")
 
 
 def conv_config_name(config: int) -> str:
@@ -337,6 +372,7 @@ class SubMIndex:
     def __init__(self, coords: torch.Tensor, stride: int = 1, table_capacity: int = 0,
                  order: str = "mask", lookup: str = "hash"):
         self.device = coords.device
+        self.order = order
         self.handle = smc_build_index(coords, stride, table_capacity, order, lookup=lookup)
         self.n, self.n_tiles = smc_get_sizes(self.handle)
 
@@ -374,14 +410,25 @@ class SubMIndex:
     def status(self) -> int:
         return smc_device_status(self.handle, self.device)
 
-    def autotune(self, feats: torch.Tensor, W: torch.Tensor, K: int = 3) -> str:
+    def autotune(self, feats: torch.Tensor, W: torch.Tensor, K: int = 3,
+                 search_orders: bool = False) -> str:
         """Choose the fastest launch configuration for this layer shape on
-        these inputs (kept for later forwards of the shape); returns its name."""
+        these inputs (kept for later forwards of the shape); with
+        search_orders the plan's row order too (for the whole handle).
+        Returns the configuration's name."""
         taps, cin, cout = W.shape
         if taps != K ** 3 or cin != feats.shape[1] or feats.shape[0] != self.n:
             raise ValueError("feats must be [N, Cin] and W [K^3, Cin, Cout]")
         out = torch.empty((self.n, cout), dtype=feats.dtype, device=feats.device)
+        if search_orders:
+            cfg, self.order = smc_autotune_ex(self.handle, feats, W, out, K, cin, cout, True)
+            return conv_config_name(cfg)
         return conv_config_name(smc_autotune(self.handle, feats, W, out, K, cin, cout))
+
+    def replan(self, order: str) -> None:
+        """Rebuild the tile plan in another row order (the map is kept)."""
+        smc_replan(self.handle, order, self.device)
+        self.order = order
 
     def forward(self, feats: torch.Tensor, W: torch.Tensor, K: int = 3,
                 out: Optional[torch.Tensor] = None, bias: Optional[torch.Tensor] = None,

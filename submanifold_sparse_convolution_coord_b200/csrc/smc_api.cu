@@ -9,6 +9,7 @@
 struct smc_index {
   int device = 0;
   int32_t stride = 1;
+  int32_t order = SMC_ORDER_MASK;  // row order of the current tile plan
   smc::Plan plan;
   // workspace of the backward passes (transposed weights, partial sums),
   // grown stream-ordered; calls on one handle are stream-ordered
@@ -149,6 +150,7 @@ int smc_build_index_ex(const int32_t* coords_dev, int64_t n, int32_t stride,
     return SMC_ERR_CUDA;
   }
   h->stride = stride;
+  h->order = order;
   const int rc = smc::build_plan(coords_dev, n, stride, cap, order, lookup,
                                  reinterpret_cast<cudaStream_t>(stream), &h->plan);
   if (rc != SMC_OK) {
@@ -193,25 +195,37 @@ int smc_forward(smc_handle_t h, const void* feats, const void* W, void* out, int
 
 const char* smc_conv_config_name(int config) { return smc::conv_config_name(config); }
 
-int smc_autotune(smc_handle_t h, const void* feats, const void* W, void* out, int K, int cin,
-                 int cout, int dtype, smc_stream_t stream, int* chosen) {
-  if (chosen) *chosen = -1;
-  const int rc = check_call(h, K, cin, cout, dtype);
+int smc_replan(smc_handle_t h, int order, smc_stream_t stream) {
+  if (!h) return SMC_ERR_INVALID;
+  if (order != SMC_ORDER_MASK && order != SMC_ORDER_INPUT && order != SMC_ORDER_GREEDY)
+    return SMC_ERR_INVALID;
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess) return SMC_ERR_CUDA;
+  if (cur != h->device) return SMC_ERR_INVALID;
+  const int rc = smc::replan(&h->plan, order, reinterpret_cast<cudaStream_t>(stream));
   if (rc != SMC_OK) return rc;
+  h->order = order;
+  h->n_tuned = 0;  // configurations were chosen for the previous plan
+  return SMC_OK;
+}
+
+namespace {
+
+// Time every valid tensor-core configuration of the shape on the caller's
+// buffers (one warm-up, best of three); *best_cfg / *best_ms get the fastest.
+int search_configs(smc_handle_t h, const void* feats, const void* W, void* out, int K, int cin,
+                   int cout, int dtype, cudaStream_t s, int* best_cfg, float* best_ms) {
   const smc::Plan& plan = h->plan;
-  if (plan.n == 0 || !smc::conv_tc_supported(cin, cout, dtype)) return SMC_OK;
-  if (!feats || !W || !out) return SMC_ERR_INVALID;
-  if (!aligned16(feats) || !aligned16(W) || !aligned16(out)) return SMC_ERR_INVALID;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool dense = K == 1;
+  *best_cfg = -1;
+  *best_ms = 0.f;
   cudaEvent_t ev[2];
   if (cudaEventCreate(&ev[0]) != cudaSuccess) return SMC_ERR_CUDA;
   if (cudaEventCreate(&ev[1]) != cudaSuccess) {
     cudaEventDestroy(ev[0]);
     return SMC_ERR_CUDA;
   }
-  int best = -1, status = SMC_OK;
-  float best_ms = 0.f;
+  int status = SMC_OK;
   const smc::Epilogue none;
   for (int cfg = 0; cfg < smc::kConvConfigs && status == SMC_OK; ++cfg) {
     if (!smc::conv_config_valid(cfg, dense, cin, cout)) continue;
@@ -228,25 +242,76 @@ int smc_autotune(smc_handle_t h, const void* feats, const void* W, void* out, in
         status = SMC_ERR_CUDA;
       if (rep == 1 || (rep > 1 && ms < t)) t = ms;  // the first run warms up
     }
-    if (status == SMC_OK && (best < 0 || t < best_ms)) {
-      best = cfg;
-      best_ms = t;
+    if (status == SMC_OK && (*best_cfg < 0 || t < *best_ms)) {
+      *best_cfg = cfg;
+      *best_ms = t;
     }
   }
   cudaEventDestroy(ev[0]);
   cudaEventDestroy(ev[1]);
   if (status != SMC_OK) return status;
   // a candidate whose bounded wait gave up leaves the choice as it was
-  status = smc_device_status(h, stream);
-  if (status != SMC_OK) return status;
-  if (best >= 0) {
-    h->set_tuned(K, cin, cout, dtype, best);
-    // leave out holding the chosen configuration's result
-    status = smc::launch_conv_tc(plan, dense, feats, W, out, cin, cout, dtype, none, s, best);
-    if (status != SMC_OK) return status;
+  return smc_device_status(h, reinterpret_cast<smc_stream_t>(s));
+}
+
+}  // namespace
+
+int smc_autotune_ex(smc_handle_t h, const void* feats, const void* W, void* out, int K, int cin,
+                    int cout, int dtype, int search_orders, smc_stream_t stream,
+                    int* chosen_config, int* chosen_order) {
+  if (chosen_config) *chosen_config = -1;
+  if (chosen_order) *chosen_order = h ? h->order : -1;
+  const int rc = check_call(h, K, cin, cout, dtype);
+  if (rc != SMC_OK) return rc;
+  const smc::Plan& plan = h->plan;
+  if (plan.n == 0 || !smc::conv_tc_supported(cin, cout, dtype)) return SMC_OK;
+  if (!feats || !W || !out) return SMC_ERR_INVALID;
+  if (!aligned16(feats) || !aligned16(W) || !aligned16(out)) return SMC_ERR_INVALID;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int best_cfg = -1, best_order = h->order;
+  float best_ms = 0.f;
+  if (search_orders && K == 3) {
+    // the row orders worth trying (the input order is an ablation)
+    const int32_t orders[2] = {SMC_ORDER_MASK, SMC_ORDER_GREEDY};
+    for (int32_t order : orders) {
+      if (order != h->order) {
+        const int r = smc_replan(h, order, stream);
+        if (r != SMC_OK) return r;
+      }
+      int cfg = -1;
+      float ms = 0.f;
+      const int r = search_configs(h, feats, W, out, K, cin, cout, dtype, s, &cfg, &ms);
+      if (r != SMC_OK) return r;
+      if (cfg >= 0 && (best_cfg < 0 || ms < best_ms)) {
+        best_cfg = cfg;
+        best_ms = ms;
+        best_order = order;
+      }
+    }
+    if (best_order != h->order) {
+      const int r = smc_replan(h, best_order, stream);
+      if (r != SMC_OK) return r;
+    }
+  } else {
+    const int r = search_configs(h, feats, W, out, K, cin, cout, dtype, s, &best_cfg, &best_ms);
+    if (r != SMC_OK) return r;
   }
-  if (chosen) *chosen = best;
+  if (best_cfg >= 0) {
+    h->set_tuned(K, cin, cout, dtype, best_cfg);
+    // leave out holding the chosen configuration's result
+    const smc::Epilogue none;
+    const int r = smc::launch_conv_tc(plan, K == 1, feats, W, out, cin, cout, dtype, none, s,
+                                      best_cfg);
+    if (r != SMC_OK) return r;
+  }
+  if (chosen_config) *chosen_config = best_cfg;
+  if (chosen_order) *chosen_order = best_order;
   return SMC_OK;
+}
+
+int smc_autotune(smc_handle_t h, const void* feats, const void* W, void* out, int K, int cin,
+                 int cout, int dtype, smc_stream_t stream, int* chosen) {
+  return smc_autotune_ex(h, feats, W, out, K, cin, cout, dtype, 0, stream, chosen, nullptr);
 }
 
 int smc_backward_input(smc_handle_t h, const void* grad_out, const void* W, void* grad_in, int K,

@@ -698,61 +698,12 @@ uint64_t table_slots(int64_t n, int64_t table_capacity) {
   return cap;
 }
 
-int build_plan_impl(const int32_t* coords, int64_t n, int32_t stride, int64_t table_capacity,
-                    int32_t order, int32_t lookup, cudaStream_t s, Plan* plan,
-                    void** scratch_mem) {
-  const bool sorted = lookup == SMC_LOOKUP_SORT;
-  const int4* c4 = reinterpret_cast<const int4*>(coords);
-  plan->n = n;
-  plan->n_tiles = (n + kTileRows - 1) / kTileRows;
-  const int64_t nt = plan->n_tiles;
-  const uint64_t cap = n > 0 ? table_slots(n, table_capacity) : 1;
-
-  // two allocations: the plan's arena (kept) and the build's scratch (freed)
-  Carve pc;
-  BuildCounters* ctr = nullptr;
-  carve_plan(pc, plan, &ctr);
-  if (dev_alloc(&plan->arena, pc.off, s) != cudaSuccess) {
-    cudaGetLastError();
-    plan->arena = nullptr;
-    return SMC_ERR_OOM;
-  }
-  pc = Carve{static_cast<uint8_t*>(plan->arena), 0};
-  carve_plan(pc, plan, &ctr);
-  plan->status = &ctr->status;
-  if (cudaMemsetAsync(ctr, 0, sizeof(BuildCounters), s) != cudaSuccess) return SMC_ERR_CUDA;
-  if (n == 0) return SMC_OK;
-
-  Carve scc;
-  Scratch sc;
-  carve_scratch(scc, &sc, n, nt, cap, sorted);
-  if (dev_alloc(scratch_mem, scc.off, s) != cudaSuccess) {
-    cudaGetLastError();
-    *scratch_mem = nullptr;
-    return SMC_ERR_OOM;
-  }
-  scc = Carve{static_cast<uint8_t*>(*scratch_mem), 0};
-  carve_scratch(scc, &sc, n, nt, cap, sorted);
-
-  // 1. lookup structure; 2. neighbour map and masks
-  if (sorted) {
-    k_pack_keys<<<grid_for(n, 256), 256, 0, s>>>(c4, n, sc.ckeys[0], sc.svals[0], plan->status);
-    SMC_LAUNCHED();
-    int cur = 0;
-    SMC_TRY(radix_sort(sc.ckeys, sc.svals, 0, n, 64, sc.hist, s, &cur));
-    k_sorted_dups<<<grid_for(n, 256), 256, 0, s>>>(sc.ckeys[cur], n, plan->status);
-    k_neighbors_sorted<<<grid_for(n, kNbrWarps), kNbrWarps * 32, 0, s>>>(
-        c4, n, stride, sc.ckeys[cur], sc.svals[cur], plan->nbr, plan->mask);
-  } else {
-    if (cudaMemsetAsync(sc.table, 0xFF, cap * sizeof(Slot), s) != cudaSuccess)
-      return SMC_ERR_CUDA;
-    const int shift = 64 - log2_pow2(cap);
-    k_insert<<<grid_for(n, 256), 256, 0, s>>>(c4, n, sc.table, cap - 1, shift, plan->status);
-    k_neighbors<<<grid_for(n, kNbrWarps), kNbrWarps * 32, 0, s>>>(c4, n, stride, sc.table, cap - 1,
-                                                                  shift, plan->nbr, plan->mask);
-  }
-  SMC_LAUNCHED();
-
+// Steps 3-5 of the build (row order, tile plan, work items) and the one
+// read-back, from the neighbour map and masks already in the plan's arena;
+// the build's counters must be zero.
+int order_and_tile(Plan* plan, BuildCounters* ctr, const Scratch& sc, int32_t order,
+                   cudaStream_t s) {
+  const int64_t n = plan->n, nt = plan->n_tiles;
   // 3. row order
   if (order == SMC_ORDER_MASK) {
     // four 8-bit passes end where they started: sort straight into perm
@@ -842,6 +793,64 @@ int build_plan_impl(const int32_t* coords, int64_t n, int32_t stride, int64_t ta
   return SMC_OK;
 }
 
+int build_plan_impl(const int32_t* coords, int64_t n, int32_t stride, int64_t table_capacity,
+                    int32_t order, int32_t lookup, cudaStream_t s, Plan* plan,
+                    void** scratch_mem) {
+  const bool sorted = lookup == SMC_LOOKUP_SORT;
+  const int4* c4 = reinterpret_cast<const int4*>(coords);
+  plan->n = n;
+  plan->n_tiles = (n + kTileRows - 1) / kTileRows;
+  const int64_t nt = plan->n_tiles;
+  const uint64_t cap = n > 0 ? table_slots(n, table_capacity) : 1;
+
+  // two allocations: the plan's arena (kept) and the build's scratch (freed)
+  Carve pc;
+  BuildCounters* ctr = nullptr;
+  carve_plan(pc, plan, &ctr);
+  if (dev_alloc(&plan->arena, pc.off, s) != cudaSuccess) {
+    cudaGetLastError();
+    plan->arena = nullptr;
+    return SMC_ERR_OOM;
+  }
+  pc = Carve{static_cast<uint8_t*>(plan->arena), 0};
+  carve_plan(pc, plan, &ctr);
+  plan->status = &ctr->status;
+  if (cudaMemsetAsync(ctr, 0, sizeof(BuildCounters), s) != cudaSuccess) return SMC_ERR_CUDA;
+  if (n == 0) return SMC_OK;
+
+  Carve scc;
+  Scratch sc;
+  carve_scratch(scc, &sc, n, nt, cap, sorted);
+  if (dev_alloc(scratch_mem, scc.off, s) != cudaSuccess) {
+    cudaGetLastError();
+    *scratch_mem = nullptr;
+    return SMC_ERR_OOM;
+  }
+  scc = Carve{static_cast<uint8_t*>(*scratch_mem), 0};
+  carve_scratch(scc, &sc, n, nt, cap, sorted);
+
+  // 1. lookup structure; 2. neighbour map and masks
+  if (sorted) {
+    k_pack_keys<<<grid_for(n, 256), 256, 0, s>>>(c4, n, sc.ckeys[0], sc.svals[0], plan->status);
+    SMC_LAUNCHED();
+    int cur = 0;
+    SMC_TRY(radix_sort(sc.ckeys, sc.svals, 0, n, 64, sc.hist, s, &cur));
+    k_sorted_dups<<<grid_for(n, 256), 256, 0, s>>>(sc.ckeys[cur], n, plan->status);
+    k_neighbors_sorted<<<grid_for(n, kNbrWarps), kNbrWarps * 32, 0, s>>>(
+        c4, n, stride, sc.ckeys[cur], sc.svals[cur], plan->nbr, plan->mask);
+  } else {
+    if (cudaMemsetAsync(sc.table, 0xFF, cap * sizeof(Slot), s) != cudaSuccess)
+      return SMC_ERR_CUDA;
+    const int shift = 64 - log2_pow2(cap);
+    k_insert<<<grid_for(n, 256), 256, 0, s>>>(c4, n, sc.table, cap - 1, shift, plan->status);
+    k_neighbors<<<grid_for(n, kNbrWarps), kNbrWarps * 32, 0, s>>>(c4, n, stride, sc.table, cap - 1,
+                                                                  shift, plan->nbr, plan->mask);
+  }
+  SMC_LAUNCHED();
+
+  return order_and_tile(plan, ctr, sc, order, s);
+}
+
 }  // namespace
 
 void free_plan(Plan* plan) {
@@ -855,6 +864,34 @@ void free_plan(Plan* plan) {
     cudaStreamSynchronize(nullptr);
   }
   *plan = Plan{};
+}
+
+int replan(Plan* plan, int32_t order, cudaStream_t s) {
+  if (plan->n == 0) return SMC_OK;
+  // a forward queued on any stream may still read the plan being rewritten
+  if (cudaDeviceSynchronize() != cudaSuccess) return SMC_ERR_CUDA;
+  // the counters sit at the start of the arena (carve_plan)
+  BuildCounters* ctr = static_cast<BuildCounters*>(plan->arena);
+  if (cudaMemsetAsync(&ctr->total_slots, 0, sizeof(BuildCounters) - sizeof(int32_t), s) !=
+      cudaSuccess)
+    return SMC_ERR_CUDA;
+  Carve scc;
+  Scratch sc;
+  carve_scratch(scc, &sc, plan->n, plan->n_tiles, 1, false);
+  void* mem = nullptr;
+  if (dev_alloc(&mem, scc.off, s) != cudaSuccess) {
+    cudaGetLastError();
+    return SMC_ERR_OOM;
+  }
+  scc = Carve{static_cast<uint8_t*>(mem), 0};
+  carve_scratch(scc, &sc, plan->n, plan->n_tiles, 1, false);
+  const int rc = order_and_tile(plan, ctr, sc, order, s);
+  dev_free(mem, s);
+  if (rc != SMC_OK) {
+    cudaGetLastError();
+    cudaStreamSynchronize(s);
+  }
+  return rc;
 }
 
 int build_plan(const int32_t* coords, int64_t n, int32_t stride, int64_t table_capacity,

@@ -73,6 +73,10 @@ struct Epilogue {
 int build_plan(const int32_t* coords, int64_t n, int32_t stride, int64_t table_capacity,
                int32_t order, int32_t lookup, cudaStream_t stream, Plan* plan);
 void free_plan(Plan* plan);
+// Rebuild the row order, tile plan and work items of a built plan in another
+// order, from its neighbour map and masks (smc_index.cu).  Waits for the
+// device first: no forward may be reading the plan.
+int replan(Plan* plan, int32_t order, cudaStream_t stream);
 
 // Tensor-core convolution (smc_conv_tc.cu).  feats/W/out in f16 or bf16.
 // dense = true runs the K = 1 form (rows in order, one tap, no plan arrays).

@@ -193,3 +193,50 @@ def test_handle_survives_errors_and_reuse():
         assert np.array_equal(m, native.neighbor_map(co))
         assert idx.status() == 0
         idx.close()
+
+
+@pytest.mark.parametrize("first,then", [("mask", "greedy"), ("greedy", "mask"), ("mask", "input")])
+def test_replan_equals_fresh_build(first, then):
+    """Rebuilding a handle's plan in another row order (from its stored map)
+    gives exactly the plan a fresh build in that order gives, and the
+    convolution over it matches the oracle."""
+    inp = synth.make_inputs("uniform64")
+    ref = native.neighbor_map(inp.coords)
+    idx, _ = _gpu_map(inp.coords, order=first)
+    idx.replan(then)
+    fresh, _ = _gpu_map(inp.coords, order=then)
+    p1, t1 = idx.tile_plan()
+    p2, t2 = fresh.tile_plan()
+    assert torch.equal(p1, p2) and torch.equal(t1, t2)
+    assert idx.plan_stats() == fresh.plan_stats()
+    assert np.array_equal(idx.neighbor_map().cpu().numpy(), ref)
+    _check_plan(idx, ref)
+    W = inp.weights[0]
+    out = idx.forward(inp.feats.to(DEV), W.to(DEV))
+    torch.cuda.synchronize()
+    assert idx.status() == 0
+    want, scale = native.submconv(inp.feats.double().numpy(), W.double().numpy(), ref)
+    from gpu_common import check_conv
+    check_conv(out, want, scale, f"replan {first} -> {then}")
+    fresh.close()
+    idx.close()
+
+
+def test_autotune_over_orders():
+    """The search over row orders and launch configurations leaves the handle
+    in one of the searched orders, with a forward that matches the oracle."""
+    inp = synth.make_inputs("uniform64")
+    ref = native.neighbor_map(inp.coords)
+    idx, _ = _gpu_map(inp.coords, order="mask")
+    W = inp.weights[0]
+    f, w = inp.feats.to(DEV), W.to(DEV)
+    name = idx.autotune(f, w, K=3, search_orders=True)
+    assert name != "cuda-cores" and idx.order in ("mask", "greedy")
+    _check_plan(idx, ref)
+    out = idx.forward(f, w)
+    torch.cuda.synchronize()
+    assert idx.status() == 0
+    want, scale = native.submconv(inp.feats.double().numpy(), W.double().numpy(), ref)
+    from gpu_common import check_conv
+    check_conv(out, want, scale, f"autotuned {idx.order} {name}")
+    idx.close()
