@@ -51,6 +51,8 @@ NCU_TRAFFIC: dict = {
     ("resblock64", 0, "greedy"): 99606784 + 32485376,
     ("resblock64", 1, "greedy"): 57634048 + 59953664,
     ("uniform64", 0, "greedy"): 4848640 + 0,
+    ("shells512", 0, "greedy"): 6102113024 + 601634048,
+    ("tiny16", 0, "greedy"): 116480 + 0,
 }
 # fp32 features run on the CUDA cores with fp64 accumulation: the ALU bound is
 # the fp64 FMA rate, 148 SMs x 64 fp64 lanes x 2 FLOP x 1.965 GHz.
