@@ -37,7 +37,10 @@
 //               issuers cover each other's loop and wait overheads;
 //   warps 2-5   epilogue: tensor memory -> registers -> fp16/bf16 -> global,
 //               overlapping the next item's MMAs when there are two
-//               accumulator sets (NBUF = 2);
+//               accumulator sets (NBUF = 2).  Where shared memory has room,
+//               each warp passes its 32 rows through a staging block so that
+//               every store writes 64-byte row pieces (8 rows per
+//               instruction) rather than 16-byte pieces of 32 rows;
 //   warp 6      index prefetcher: lane 0 bulk-copies the 128 gather indices
 //               of each A unit into a ring of index blocks, running up to a
 //               full ring of units ahead of the gathers;
@@ -270,6 +273,31 @@ __device__ __forceinline__ int index_slot(const Item<G>& it, int k, int t) {
   return it.slot0[k] + __popc(it.mask[k] & ((1u << t) - 1u));
 }
 
+// Shared-memory layout: A ring, W ring, index ring (the rings), then the
+// barriers and the small per-CTA state (the tail), then, when the rings leave
+// room for it, the epilogue's output staging: per epilogue warp 32 rows of 32
+// output columns, each row's 64 bytes padded to 80 so that both the row-wise
+// writes and the column-wise reads are free of bank conflicts.
+constexpr int kStageRowBytes = 80;
+constexpr int kStageBytes = 4 * 32 * kStageRowBytes;
+template <int BN, int NA, int NW, int KS, bool PAIR>
+__host__ __device__ constexpr int smem_rings() {
+  return NA * (KS * kSubBytes + (PAIR ? 2 : 1) * kIdxBytes) + NW * KS * BN * kBK * 2;
+}
+template <int NA, int NW, int G>
+__host__ __device__ constexpr int smem_tail() {
+  return ((4 * NA + 2 * NW + 8) * 8 + 2 * int(sizeof(Item<G>)) + 16 + 15) & ~15;
+}
+template <int BN, int NA, int NW, int G, int KS, bool PAIR>
+__host__ __device__ constexpr bool staged_output() {
+  return smem_rings<BN, NA, NW, KS, PAIR>() + smem_tail<NA, NW, G>() + kStageBytes <= 227 * 1024;
+}
+template <int BN, int NA, int NW, int G, int KS, bool PAIR>
+__host__ __device__ constexpr int smem_bytes() {
+  return smem_rings<BN, NA, NW, KS, PAIR>() + smem_tail<NA, NW, G>() +
+         (staged_output<BN, NA, NW, G, KS, PAIR>() ? kStageBytes : 0);
+}
+
 // NA: A units in flight (16 KS KB each), NW: W slices in flight, NQ gather
 // groups of WPS warps, NBUF accumulator sets in tensor memory (2: the epilogue
 // of one item overlaps the MMAs of the next; 1: room for two 256-column
@@ -322,9 +350,11 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
   // barriers: afull[NA] aempty[NA] ifull[NA] iempty[NA] wfull[NW] wempty[NW]
   //           tfull[2] tempty[2] info[2] drain[2]
   constexpr int kBars = 4 * NA + 2 * NW + 6 + 2;
+  constexpr bool kStaged = staged_output<BN, NA, NW, G, KS, PAIR>();
   Item<G>* acc_info = reinterpret_cast<Item<G>*>(bars + kBars);  // item of each accumulator set
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_info + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint8_t* out_stage = smem_raw + smem_rings<BN, NA, NW, KS, PAIR>() + smem_tail<NA, NW, G>();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kb_per_tap = PAIR ? 1 : args.cin / (kBK * KS);  // stages per tap (pair)
@@ -707,6 +737,35 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
           uint32_t v[32];
           tmem_ld_x32(tmem + (uint32_t(quarter * 32) << 16) + (a * G + k) * BN + uint32_t(cc * 32),
                       v);
+          if constexpr (kStaged) {
+            // this lane's row piece into the warp's staging rows, then each
+            // store writes 64-byte pieces of 8 rows (4 lanes per row)
+            if (orow[k] >= 0 && (args.bias || args.residual || args.act != SMC_ACT_NONE))
+              apply_epilogue<BF16>(v, args, orow[k], it.n0 + cc * 32);
+            uint8_t* st_rows = out_stage + quarter * (32 * kStageRowBytes);
+            uint4* mine_row = reinterpret_cast<uint4*>(st_rows + lane * kStageRowBytes);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint4 o;
+              o.x = pack2<BF16>(v[8 * q + 0], v[8 * q + 1]);
+              o.y = pack2<BF16>(v[8 * q + 2], v[8 * q + 3]);
+              o.z = pack2<BF16>(v[8 * q + 4], v[8 * q + 5]);
+              o.w = pack2<BF16>(v[8 * q + 6], v[8 * q + 7]);
+              mine_row[q] = o;
+            }
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int r = 8 * i + (lane >> 2), c = lane & 3;
+              const int32_t orr = __shfl_sync(0xffffffffu, orow[k], r);
+              const uint4 val = *reinterpret_cast<const uint4*>(st_rows + r * kStageRowBytes + c * 16);
+              if (orr >= 0)
+                *reinterpret_cast<uint4*>(args.out + int64_t(orr) * args.cout + it.n0 + cc * 32 +
+                                          c * 8) = val;
+            }
+            __syncwarp();  // the rows are read before the next chunk overwrites them
+            continue;
+          }
           if (orow[k] >= 0) {
             if (args.bias || args.residual || args.act != SMC_ACT_NONE)
               apply_epilogue<BF16>(v, args, orow[k], it.n0 + cc * 32);
@@ -791,11 +850,7 @@ template <int BN, int NA, int NW, int G, int WPS, int NQ, bool BF16, int NBUF, i
           bool PAIR = false>
 int launch_cfg(const Plan& plan, bool dense, const void* feats, const void* W, void* out, int cin,
                int cout, const Epilogue& ep, cudaStream_t stream) {
-  constexpr int kWBytes = BN * kBK * 2;
-  constexpr int kBars = 4 * NA + 2 * NW + 6 + 2;
-  constexpr int kTail = kBars * 8 + 2 * int(sizeof(Item<G>)) + 16;
-  constexpr int kSmem =
-      NA * (KS * kSubBytes + (PAIR ? 2 : 1) * kIdxBytes) + NW * KS * kWBytes + kTail;
+  constexpr int kSmem = smem_bytes<BN, NA, NW, G, KS, PAIR>();
   static_assert(kSmem <= 227 * 1024, "shared memory");
   static_assert(threads_for(NQ, WPS) <= 1024, "threads");
   auto kern = k_conv_tc<BN, NA, NW, G, WPS, NQ, BF16, NBUF, KS, PAIR>;
