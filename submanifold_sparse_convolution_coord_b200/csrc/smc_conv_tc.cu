@@ -302,8 +302,10 @@ __host__ __device__ constexpr int smem_bytes() {
 // groups of WPS warps, NBUF accumulator sets in tensor memory (2: the epilogue
 // of one item overlaps the MMAs of the next; 1: room for two 256-column
 // tiles), KS: 64-channel sub-chunks per unit, PAIR: the two sub-chunks are
-// two taps of 64-channel rows (else KS chunks of one tap).
-template <int BN, int NA, int NW, int G, int WPS, int NQ, bool BF16, int NBUF, int KS, bool PAIR>
+// two taps of 64-channel rows (else KS chunks of one tap), EPI: the fused
+// epilogue (bias, activation, residual) is applied.
+template <int BN, int NA, int NW, int G, int WPS, int NQ, bool BF16, int NBUF, int KS, bool PAIR,
+          bool EPI>
 __global__ void __launch_bounds__(threads_for(NQ, WPS), 1)
 k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap fmap,
           const ConvArgs args) {
@@ -740,8 +742,7 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
           if constexpr (kStaged) {
             // this lane's row piece into the warp's staging rows, then each
             // store writes 64-byte pieces of 8 rows (4 lanes per row)
-            if (orow[k] >= 0 && (args.bias || args.residual || args.act != SMC_ACT_NONE))
-              apply_epilogue<BF16>(v, args, orow[k], it.n0 + cc * 32);
+            if (EPI && orow[k] >= 0) apply_epilogue<BF16>(v, args, orow[k], it.n0 + cc * 32);
             uint8_t* st_rows = out_stage + quarter * (32 * kStageRowBytes);
             uint4* mine_row = reinterpret_cast<uint4*>(st_rows + lane * kStageRowBytes);
 #pragma unroll
@@ -767,8 +768,7 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
             continue;
           }
           if (orow[k] >= 0) {
-            if (args.bias || args.residual || args.act != SMC_ACT_NONE)
-              apply_epilogue<BF16>(v, args, orow[k], it.n0 + cc * 32);
+            if (EPI) apply_epilogue<BF16>(v, args, orow[k], it.n0 + cc * 32);
             uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -847,13 +847,13 @@ bool encode_2d(CUtensorMap* map, bool bf16, const void* base, uint64_t cols, uin
 }
 
 template <int BN, int NA, int NW, int G, int WPS, int NQ, bool BF16, int NBUF, int KS,
-          bool PAIR = false>
+          bool PAIR, bool EPI>
 int launch_cfg(const Plan& plan, bool dense, const void* feats, const void* W, void* out, int cin,
                int cout, const Epilogue& ep, cudaStream_t stream) {
   constexpr int kSmem = smem_bytes<BN, NA, NW, G, KS, PAIR>();
   static_assert(kSmem <= 227 * 1024, "shared memory");
   static_assert(threads_for(NQ, WPS) <= 1024, "threads");
-  auto kern = k_conv_tc<BN, NA, NW, G, WPS, NQ, BF16, NBUF, KS, PAIR>;
+  auto kern = k_conv_tc<BN, NA, NW, G, WPS, NQ, BF16, NBUF, KS, PAIR, EPI>;
   // the shared-memory limit is a per-device function attribute: set it once
   // on each device this configuration runs on
   constexpr int kMaxDev = 64;
@@ -912,19 +912,24 @@ int group_override() {
 template <bool BF16>
 int launch_config(int cfg, const Plan& plan, bool dense, const void* feats, const void* W,
                   void* out, int cin, int cout, const Epilogue& ep, cudaStream_t stream) {
-#define SMC_CFG(...) return launch_cfg<__VA_ARGS__>(plan, dense, feats, W, out, cin, cout, ep, stream)
+  // the fused epilogue (bias, activation, residual) is its own instantiation,
+  // so the plain convolution carries none of its code
+  const bool epi = ep.bias || ep.residual || ep.act != SMC_ACT_NONE;
+#define SMC_CFG(...)                                                                         \
+  return epi ? launch_cfg<__VA_ARGS__, true>(plan, dense, feats, W, out, cin, cout, ep, stream) \
+             : launch_cfg<__VA_ARGS__, false>(plan, dense, feats, W, out, cin, cout, ep, stream)
   switch (cfg) {  //            BN  NA NW G WPS NQ        NBUF KS PAIR
-    case kCfg256G2: SMC_CFG(256, 9, 2, 2, 4, 3, BF16, 1, 1);
-    case kCfg256G1: SMC_CFG(256, 9, 2, 1, 4, 3, BF16, 2, 1);
-    case kCfg256G1K2: SMC_CFG(256, 3, 2, 1, 4, 3, BF16, 2, 2);
-    case kCfg128G2K2: SMC_CFG(128, 4, 2, 2, 4, 2, BF16, 2, 2);
-    case kCfg128G1K2: SMC_CFG(128, 4, 2, 1, 4, 2, BF16, 2, 2);
+    case kCfg256G2: SMC_CFG(256, 9, 2, 2, 4, 3, BF16, 1, 1, false);
+    case kCfg256G1: SMC_CFG(256, 9, 2, 1, 4, 3, BF16, 2, 1, false);
+    case kCfg256G1K2: SMC_CFG(256, 2, 2, 1, 4, 2, BF16, 2, 2, false);
+    case kCfg128G2K2: SMC_CFG(128, 4, 2, 2, 4, 2, BF16, 2, 2, false);
+    case kCfg128G1K2: SMC_CFG(128, 4, 2, 1, 4, 2, BF16, 2, 2, false);
     case kCfg128G1Pair: SMC_CFG(128, 4, 2, 1, 4, 2, BF16, 2, 2, true);
-    case kCfg128G2: SMC_CFG(128, 10, 3, 2, 2, 5, BF16, 2, 1);
-    case kCfg128G1: SMC_CFG(128, 10, 3, 1, 2, 5, BF16, 2, 1);
+    case kCfg128G2: SMC_CFG(128, 10, 3, 2, 2, 5, BF16, 2, 1, false);
+    case kCfg128G1: SMC_CFG(128, 10, 3, 1, 2, 5, BF16, 2, 1, false);
     case kCfg64G1Pair: SMC_CFG(64, 5, 2, 1, 2, 5, BF16, 2, 2, true);
-    case kCfg64G2: SMC_CFG(64, 12, 3, 2, 2, 6, BF16, 2, 1);
-    case kCfg64G1: SMC_CFG(64, 12, 3, 1, 2, 6, BF16, 2, 1);
+    case kCfg64G2: SMC_CFG(64, 12, 3, 2, 2, 6, BF16, 2, 1, false);
+    case kCfg64G1: SMC_CFG(64, 12, 3, 1, 2, 6, BF16, 2, 1, false);
     default: return SMC_ERR_INVALID;
   }
 #undef SMC_CFG
