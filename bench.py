@@ -47,11 +47,10 @@ DTYPE_NAME = {"f16": "f16", "bf16": "bf16", "f32": "f32"}
 # launch (bytes; profiles/k_conv_tc_*.md).  Cases not captured with the current
 # kernel report null.
 NCU_TRAFFIC: dict = {
-    ("uniform128", 0, "greedy"): 64355584 + 14522624,
-    ("resblock64", 0, "greedy"): 99606784 + 32485376,
-    ("resblock64", 1, "greedy"): 57634048 + 59953664,
-    ("uniform64", 0, "greedy"): 4848640 + 0,
-    ("shells512", 0, "greedy"): 6102113024 + 601634048,
+    ("uniform128", 0, "greedy"): 65614592 + 20199680,
+    ("resblock64", 0, "greedy"): 105441536 + 35173632,
+    ("resblock64", 1, "greedy"): 57596672 + 60187392,
+    ("uniform64", 0, "greedy"): 4823808 + 0,
     ("tiny16", 0, "greedy"): 116480 + 0,
 }
 # fp32 features run on the CUDA cores with fp64 accumulation: the ALU bound is
