@@ -40,7 +40,9 @@
 //               accumulator sets (NBUF = 2).  Where shared memory has room,
 //               each warp passes its 32 rows through a staging block so that
 //               every store writes 64-byte row pieces (8 rows per
-//               instruction) rather than 16-byte pieces of 32 rows;
+//               instruction) rather than 16-byte pieces of 32 rows.  The
+//               CTA's last item is stored together with the first four
+//               gather warps, which are idle by then;
 //   warp 6      index prefetcher: lane 0 bulk-copies the 128 gather indices
 //               of each A unit into a ring of index blocks, running up to a
 //               full ring of units ahead of the gathers;
@@ -286,7 +288,7 @@ __host__ __device__ constexpr int smem_rings() {
 }
 template <int NA, int NW, int G>
 __host__ __device__ constexpr int smem_tail() {
-  return ((4 * NA + 2 * NW + 8) * 8 + 2 * int(sizeof(Item<G>)) + 16 + 15) & ~15;
+  return ((4 * NA + 2 * NW + 9) * 8 + 2 * int(sizeof(Item<G>)) + 16 + 15) & ~15;
 }
 template <int BN, int NA, int NW, int G, int KS, bool PAIR>
 __host__ __device__ constexpr bool staged_output() {
@@ -350,8 +352,8 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
   int32_t* idx_ring = reinterpret_cast<int32_t*>(w_ring + NW * kWStage);  // NA x kIdxSlot
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(idx_ring) + NA * kIdxSlot);
   // barriers: afull[NA] aempty[NA] ifull[NA] iempty[NA] wfull[NW] wempty[NW]
-  //           tfull[2] tempty[2] info[2] drain[2]
-  constexpr int kBars = 4 * NA + 2 * NW + 6 + 2;
+  //           tfull[2] tempty[2] info[2] drain[2] lastdone
+  constexpr int kBars = 4 * NA + 2 * NW + 6 + 2 + 1;
   constexpr bool kStaged = staged_output<BN, NA, NW, G, KS, PAIR>();
   Item<G>* acc_info = reinterpret_cast<Item<G>*>(bars + kBars);  // item of each accumulator set
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_info + 2);
@@ -371,6 +373,7 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
   const uint32_t tempty0 = tfull0 + 16;
   const uint32_t info0 = tempty0 + 16;
   const uint32_t drain0 = info0 + 16;
+  const uint32_t lastdone = drain0 + 16;  // the CTA's last item's MMAs are done
   const uint32_t a_base = smem_addr(a_ring);
   const uint32_t w_base = smem_addr(w_ring);
   const uint32_t i_base = smem_addr(idx_ring);
@@ -394,6 +397,7 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
       mbar_init(info0 + 8 * a, 1);
       mbar_init(drain0 + 8 * a, 1);
     }
+    mbar_init(lastdone, kMmaWarps);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -420,6 +424,80 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
     return it;
   };
   auto first_record = [&]() { return item_record(args, item_of(0, total_work)); };
+
+  // Epilogue pieces, used by the epilogue warps and, for the CTA's last item,
+  // by the first four gather warps.  A warp handles the tensor-memory lanes
+  // (rows) 32 * (warp % 4) ... + 31 of every tile of the item.
+  constexpr int kChunks = BN / 32;  // 32-column chunks of a tile
+  auto output_rows = [&](const Item<G>& it, int32_t (&orow)[G]) {
+    const int row = (warp & 3) * 32 + lane;
+#pragma unroll
+    for (int k = 0; k < G; ++k) {
+      const int64_t r = int64_t(it.tile0 + k) * kTileRows + row;
+      if (it.mask[k] == 0)
+        orow[k] = -1;
+      else if (args.dense)
+        orow[k] = r < args.n ? int32_t(r) : -1;
+      else
+        orow[k] = args.out_row[r];
+    }
+  };
+  // Chunks cc0 .. cc1 - 1 of every tile of the item in accumulator set a.
+  auto store_columns = [&](const Item<G>& it, uint32_t a, const int32_t (&orow)[G], int cc0,
+                           int cc1, uint8_t* st_rows) {
+    const int quarter = warp & 3;
+#pragma unroll
+    for (int k = 0; k < G; ++k) {
+      if (it.mask[k] == 0) continue;  // past the last tile
+      uint16_t* dst = args.out + int64_t(orow[k] < 0 ? 0 : orow[k]) * args.cout + it.n0;
+#pragma unroll 1
+      for (int cc = cc0; cc < cc1; ++cc) {
+        uint32_t v[32];
+        tmem_ld_x32(tmem + (uint32_t(quarter * 32) << 16) + (a * G + k) * BN + uint32_t(cc * 32),
+                    v);
+        if constexpr (kStaged) {
+          // this lane's row piece into the warp's staging rows, then each
+          // store writes 64-byte pieces of 8 rows (4 lanes per row)
+          if (EPI && orow[k] >= 0) apply_epilogue<BF16>(v, args, orow[k], it.n0 + cc * 32);
+          uint4* mine_row = reinterpret_cast<uint4*>(st_rows + lane * kStageRowBytes);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 o;
+            o.x = pack2<BF16>(v[8 * q + 0], v[8 * q + 1]);
+            o.y = pack2<BF16>(v[8 * q + 2], v[8 * q + 3]);
+            o.z = pack2<BF16>(v[8 * q + 4], v[8 * q + 5]);
+            o.w = pack2<BF16>(v[8 * q + 6], v[8 * q + 7]);
+            mine_row[q] = o;
+          }
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int r = 8 * i + (lane >> 2), c = lane & 3;
+            const int32_t orr = __shfl_sync(0xffffffffu, orow[k], r);
+            const uint4 val = *reinterpret_cast<const uint4*>(st_rows + r * kStageRowBytes + c * 16);
+            if (orr >= 0)
+              *reinterpret_cast<uint4*>(args.out + int64_t(orr) * args.cout + it.n0 + cc * 32 +
+                                        c * 8) = val;
+          }
+          __syncwarp();  // the rows are read before the next chunk overwrites them
+          continue;
+        }
+        if (orow[k] >= 0) {
+          if (EPI) apply_epilogue<BF16>(v, args, orow[k], it.n0 + cc * 32);
+          uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 o;
+            o.x = pack2<BF16>(v[8 * q + 0], v[8 * q + 1]);
+            o.y = pack2<BF16>(v[8 * q + 2], v[8 * q + 3]);
+            o.z = pack2<BF16>(v[8 * q + 4], v[8 * q + 5]);
+            o.w = pack2<BF16>(v[8 * q + 6], v[8 * q + 7]);
+            d4[q] = o;
+          }
+        }
+      }
+    }
+  };
 
   if (warp == kLoaderWarp) {
     // ---------------- W loader ----------------
@@ -528,9 +606,13 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
     int4 rec = first_record();
     int last_dense = -1;  // last unit this group TMA-loaded (dense mode)
     bool ok = true;
+    Item<G> last_it;
+    uint32_t n_items = 0;
     while (ok) {
       const Item<G> it = next_item(j, rec);
       if (it.w < 0) break;
+      last_it = it;
+      ++n_items;
       uint32_t rem = rotate_taps(it.all, it.rot);
       while (rem && ok) {
         const StageTaps st = next_stage_taps<PAIR>(rem, it.rot);
@@ -607,6 +689,20 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
       }
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
+    if (ok && n_items > 0 && warp - kFirstGatherWarp < 4) {
+      // help store the CTA's last item (the second half of its columns) once
+      // its MMAs are done; the A ring is free by then and holds the staging rows
+      const uint32_t a = (n_items - 1) % NBUF;
+      int32_t orow[G];
+      output_rows(last_it, orow);
+      // one phase only, so the wait cannot mistake an earlier item for it
+      const bool have = wt.wait(lastdone, 0);
+      if (__all_sync(0xffffffffu, have)) {
+        tc_fence_after();
+        store_columns(last_it, a, orow, kChunks / 2, kChunks,
+                      a_ring + (warp & 3) * (32 * kStageRowBytes));
+      }
+    }
     if (last_dense >= 0) {
       // TMA loads this lane issued that may not have landed: the latest unit
       // of each of the group's NA / NQ slots (earlier ones were consumed)
@@ -698,6 +794,7 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
       }
       if (!ok) break;
       umma_commit(tfull0 + 8 * a);
+      if (item_of(j, total_work) < 0) umma_commit(lastdone);
       ++acc_iter;
     }
     // every MMA this warp issued completes before tensor memory and the
@@ -706,8 +803,6 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
     mbar_drain(drain0 + 8 * mine, 0);
   } else {
     // ---------------- epilogue (warps 2-5) ----------------
-    const int quarter = warp & 3;  // tensor-memory lanes 32*quarter .. +31
-    const int row = quarter * 32 + lane;
     uint32_t acc_iter = 0;
     while (true) {
       const uint32_t a = acc_iter % NBUF;
@@ -717,77 +812,20 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
       const Item<G> it = acc_info[a];
       if (it.w < 0) break;
       int32_t orow[G];
-#pragma unroll
-      for (int k = 0; k < G; ++k) {
-        const int64_t r = int64_t(it.tile0 + k) * kTileRows + row;
-        if (it.mask[k] == 0)
-          orow[k] = -1;
-        else if (args.dense)
-          orow[k] = r < args.n ? int32_t(r) : -1;
-        else
-          orow[k] = args.out_row[r];
-      }
+      output_rows(it, orow);
       have = wt.wait(tfull0 + 8 * a, use & 1);
       if (!__all_sync(0xffffffffu, have)) break;  // tcgen05.ld below is warp-collective
       tc_fence_after();
-#pragma unroll
-      for (int k = 0; k < G; ++k) {
-        if (it.mask[k] == 0) continue;  // past the last tile
-        uint16_t* dst = args.out + int64_t(orow[k] < 0 ? 0 : orow[k]) * args.cout + it.n0;
-#pragma unroll 1
-        for (int cc = 0; cc < BN / 32; ++cc) {
-          uint32_t v[32];
-          tmem_ld_x32(tmem + (uint32_t(quarter * 32) << 16) + (a * G + k) * BN + uint32_t(cc * 32),
-                      v);
-          if constexpr (kStaged) {
-            // this lane's row piece into the warp's staging rows, then each
-            // store writes 64-byte pieces of 8 rows (4 lanes per row)
-            if (EPI && orow[k] >= 0) apply_epilogue<BF16>(v, args, orow[k], it.n0 + cc * 32);
-            uint8_t* st_rows = out_stage + quarter * (32 * kStageRowBytes);
-            uint4* mine_row = reinterpret_cast<uint4*>(st_rows + lane * kStageRowBytes);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint4 o;
-              o.x = pack2<BF16>(v[8 * q + 0], v[8 * q + 1]);
-              o.y = pack2<BF16>(v[8 * q + 2], v[8 * q + 3]);
-              o.z = pack2<BF16>(v[8 * q + 4], v[8 * q + 5]);
-              o.w = pack2<BF16>(v[8 * q + 6], v[8 * q + 7]);
-              mine_row[q] = o;
-            }
-            __syncwarp();
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int r = 8 * i + (lane >> 2), c = lane & 3;
-              const int32_t orr = __shfl_sync(0xffffffffu, orow[k], r);
-              const uint4 val = *reinterpret_cast<const uint4*>(st_rows + r * kStageRowBytes + c * 16);
-              if (orr >= 0)
-                *reinterpret_cast<uint4*>(args.out + int64_t(orr) * args.cout + it.n0 + cc * 32 +
-                                          c * 8) = val;
-            }
-            __syncwarp();  // the rows are read before the next chunk overwrites them
-            continue;
-          }
-          if (orow[k] >= 0) {
-            if (EPI) apply_epilogue<BF16>(v, args, orow[k], it.n0 + cc * 32);
-            uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint4 o;
-              o.x = pack2<BF16>(v[8 * q + 0], v[8 * q + 1]);
-              o.y = pack2<BF16>(v[8 * q + 2], v[8 * q + 3]);
-              o.z = pack2<BF16>(v[8 * q + 4], v[8 * q + 5]);
-              o.w = pack2<BF16>(v[8 * q + 6], v[8 * q + 7]);
-              d4[q] = o;
-            }
-          }
-        }
-      }
+      // the CTA's last item: the second half of the columns is stored by the
+      // first four gather warps, which have nothing left to do
+      const bool last = item_of(acc_iter + 1, total_work) < 0;
+      store_columns(it, a, orow, 0, last ? kChunks / 2 : kChunks,
+                    out_stage + (warp & 3) * (32 * kStageRowBytes));
       tc_fence_before();
       mbar_arrive(tempty0 + 8 * a);
       ++acc_iter;
     }
   }
-
   tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarp) {
