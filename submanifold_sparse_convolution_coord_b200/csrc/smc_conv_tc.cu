@@ -966,8 +966,8 @@ int launch_config(int cfg, const Plan& plan, bool dense, const void* feats, cons
     case kCfg128G2: SMC_CFG(128, 10, 3, 2, 2, 5, BF16, 2, 1, false);
     case kCfg128G1: SMC_CFG(128, 10, 3, 1, 2, 5, BF16, 2, 1, false);
     case kCfg64G1Pair: SMC_CFG(64, 5, 2, 1, 2, 5, BF16, 2, 2, true);
-    case kCfg64G2: SMC_CFG(64, 12, 3, 2, 2, 6, BF16, 2, 1, false);
-    case kCfg64G1: SMC_CFG(64, 12, 3, 1, 2, 6, BF16, 2, 1, false);
+    case kCfg64G2: SMC_CFG(64, 12, 2, 2, 2, 6, BF16, 2, 1, false);
+    case kCfg64G1: SMC_CFG(64, 12, 2, 1, 2, 6, BF16, 2, 1, false);
     default: return SMC_ERR_INVALID;
   }
 #undef SMC_CFG
