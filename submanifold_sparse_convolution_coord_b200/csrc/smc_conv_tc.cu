@@ -699,6 +699,9 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
       const bool have = wt.wait(lastdone, 0);
       if (__all_sync(0xffffffffu, have)) {
         tc_fence_after();
+        // the A ring was last written by copies and read by the tensor core
+        // (async proxy); order that before these staging writes
+        fence_proxy_async_smem();
         store_columns(last_it, a, orow, kChunks / 2, kChunks,
                       a_ring + (warp & 3) * (32 * kStageRowBytes));
       }
