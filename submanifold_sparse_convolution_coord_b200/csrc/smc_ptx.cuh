@@ -47,6 +47,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// The spinning part of a bounded wait, out of line: it runs only when the
+// first try_wait fails, and keeping one copy of it rather than one per wait
+// site keeps the kernels small (they are instruction-fetch sensitive).
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity,
+                                                   volatile int* abort_flag, int32_t* status,
+                                                   uint64_t limit_ns) {
+  const uint64_t t0 = global_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (global_ns() - t0 > limit_ns) {
+      *abort_flag = 1;
+      atomicOr(status, kDevTimeout);
+      return false;
+    }
+  }
+  return true;
+}
 // Shared state of the bounded waits: the CTA's abort flag, the handle's status
 // word and the wait limit.
 struct Waits {
@@ -58,21 +75,12 @@ struct Waits {
   // CTA has already aborted.
   __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity) const {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_ns();
-    while (!mbar_try_wait(bar, parity)) {
-      if (*abort_flag) return false;
-      if (global_ns() - t0 > limit_ns) {
-        *abort_flag = 1;
-        atomicOr(status, kDevTimeout);
-        return false;
-      }
-    }
-    return true;
+    return mbar_wait_slow(bar, parity, abort_flag, status, limit_ns);
   }
 };
 // Bounded wait that ignores the abort flag: the abort path uses it to let
 // copies and MMAs already issued finish before their memory is released.
-__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
+static __device__ __noinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
   const uint64_t t0 = global_ns();
   while (!mbar_try_wait(bar, parity) && global_ns() - t0 < kDrainLimitNs) {
   }
