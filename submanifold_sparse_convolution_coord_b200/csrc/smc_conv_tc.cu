@@ -192,18 +192,19 @@ __device__ __forceinline__ int item_of(uint32_t j, int total) {
   return w < total ? int(w) : -1;
 }
 // The 16-byte record of item w (sparse mode), loaded one item ahead of use.
+template <bool DENSE>
 __device__ __forceinline__ int4 item_record(const ConvArgs& a, int w) {
-  if (w < 0 || a.dense) return make_int4(0, 0, 0, 0);
+  if (w < 0 || DENSE) return make_int4(0, 0, 0, 0);
   return __ldg(a.items + w / a.n_blocks);
 }
 
-template <int BN, int G>
+template <int BN, int G, bool DENSE>
 __device__ __forceinline__ Item<G> decode_item(const ConvArgs& a, int w, int4 r) {
   Item<G> it;
   it.w = w;
   const int q = w / a.n_blocks;
   it.n0 = (w - q * a.n_blocks) * BN;
-  if (a.dense) {
+  if constexpr (DENSE) {
     it.tile0 = q * G;
 #pragma unroll
     for (int k = 0; k < G; ++k) {
@@ -305,9 +306,11 @@ __host__ __device__ constexpr int smem_bytes() {
 // of one item overlaps the MMAs of the next; 1: room for two 256-column
 // tiles), KS: 64-channel sub-chunks per unit, PAIR: the two sub-chunks are
 // two taps of 64-channel rows (else KS chunks of one tap), EPI: the fused
-// epilogue (bias, activation, residual) is applied.
+// epilogue (bias, activation, residual) is applied, DENSE: K = 1 (contiguous
+// rows loaded by TMA, one tap, no plan arrays); each is its own instantiation
+// so that a kernel carries only the code it runs.
 template <int BN, int NA, int NW, int G, int WPS, int NQ, bool BF16, int NBUF, int KS, bool PAIR,
-          bool EPI>
+          bool EPI, bool DENSE>
 __global__ void __launch_bounds__(threads_for(NQ, WPS), 1)
 k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap fmap,
           const ConvArgs args) {
@@ -382,7 +385,7 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
     for (int s = 0; s < NA; ++s) {
       // sparse: every lane of the unit's gather group; dense: the lane that
       // TMA-loads the contiguous rows
-      mbar_init(afull0 + 8 * s, args.dense ? 1 : WPS * 32);
+      mbar_init(afull0 + 8 * s, DENSE ? 1 : WPS * 32);
       mbar_init(aempty0 + 8 * s, 1);
       mbar_init(ifull0 + 8 * s, 1);
       mbar_init(iempty0 + 8 * s, WPS);
@@ -418,12 +421,12 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
       it.w = -1;
       return it;
     }
-    it = decode_item<BN, G>(args, w, rec);
+    it = decode_item<BN, G, DENSE>(args, w, rec);
     ++j;
-    rec = item_record(args, item_of(j, total_work));
+    rec = item_record<DENSE>(args, item_of(j, total_work));
     return it;
   };
-  auto first_record = [&]() { return item_record(args, item_of(0, total_work)); };
+  auto first_record = [&]() { return item_record<DENSE>(args, item_of(0, total_work)); };
 
   // Epilogue pieces, used by the epilogue warps and, for the CTA's last item,
   // by the first four gather warps.  A warp handles the tensor-memory lanes
@@ -436,7 +439,7 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
       const int64_t r = int64_t(it.tile0 + k) * kTileRows + row;
       if (it.mask[k] == 0)
         orow[k] = -1;
-      else if (args.dense)
+      else if (DENSE)
         orow[k] = r < args.n ? int32_t(r) : -1;
       else
         orow[k] = args.out_row[r];
@@ -551,7 +554,7 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
       while (ok) {
         const Item<G> it = next_item(j, rec);
         if (it.w < 0) break;
-        if (args.dense) continue;  // K = 1 has no gather index
+        if (DENSE) continue;  // K = 1 has no gather index
         uint32_t rem = rotate_taps(it.all, it.rot);
         while (rem && ok) {
           const StageTaps st = next_stage_taps<PAIR>(rem, it.rot);
@@ -601,7 +604,7 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
     const int chunk = lane & 7;   // 16-byte chunk of a 128-byte row
     const int rsub = lane >> 3;   // instruction i copies rows 4 i + rsub of the warp's share
     const int row0 = kRowsPerWarp * wq;
-    if (args.dense && wq == 0 && lane == 0) tma_prefetch_map(&fmap);
+    if (DENSE && wq == 0 && lane == 0) tma_prefetch_map(&fmap);
     uint32_t u = 0, j = 0;
     int4 rec = first_record();
     int last_dense = -1;  // last unit this group TMA-loaded (dense mode)
@@ -625,7 +628,7 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
             if (int(my % NQ) != grp) continue;
             const uint32_t slot = my % NA, ph = (my / NA) & 1;
             const uint32_t dst = a_base + slot * kAUnitBytes;
-            if (args.dense) {
+            if constexpr (DENSE) {
               if (wq == 0 && lane == 0) {
                 if (!wt.wait(aempty0 + 8 * slot, ph ^ 1)) {
                   ok = false;
@@ -771,7 +774,7 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
             }
             // the rows were written by cp.async (generic proxy) or TMA: order
             // them before the tensor core's (async-proxy) reads
-            if (!args.dense) fence_proxy_async_smem();
+            if (!DENSE) fence_proxy_async_smem();
             tc_fence_after();
             // descriptors: the start-address field (bits 0-13, 16-byte units)
             // never carries, so byte offsets add to the 64-bit value
@@ -888,13 +891,14 @@ bool encode_2d(CUtensorMap* map, bool bf16, const void* base, uint64_t cols, uin
 }
 
 template <int BN, int NA, int NW, int G, int WPS, int NQ, bool BF16, int NBUF, int KS,
-          bool PAIR, bool EPI>
+          bool PAIR, bool EPI, bool DENSE>
 int launch_cfg(const Plan& plan, bool dense, const void* feats, const void* W, void* out, int cin,
                int cout, const Epilogue& ep, cudaStream_t stream) {
   constexpr int kSmem = smem_bytes<BN, NA, NW, G, KS, PAIR>();
   static_assert(kSmem <= 227 * 1024, "shared memory");
   static_assert(threads_for(NQ, WPS) <= 1024, "threads");
-  auto kern = k_conv_tc<BN, NA, NW, G, WPS, NQ, BF16, NBUF, KS, PAIR, EPI>;
+  static_assert(!(PAIR && DENSE), "tap pairs exist for K = 3 only");
+  auto kern = k_conv_tc<BN, NA, NW, G, WPS, NQ, BF16, NBUF, KS, PAIR, EPI, DENSE>;
   // the shared-memory limit is a per-device function attribute: set it once
   // on each device this configuration runs on
   constexpr int kMaxDev = 64;
@@ -956,24 +960,38 @@ int launch_config(int cfg, const Plan& plan, bool dense, const void* feats, cons
   // the fused epilogue (bias, activation, residual) is its own instantiation,
   // so the plain convolution carries none of its code
   const bool epi = ep.bias || ep.residual || ep.act != SMC_ACT_NONE;
-#define SMC_CFG(...)                                                                         \
-  return epi ? launch_cfg<__VA_ARGS__, true>(plan, dense, feats, W, out, cin, cout, ep, stream) \
-             : launch_cfg<__VA_ARGS__, false>(plan, dense, feats, W, out, cin, cout, ep, stream)
+#define SMC_CFG(...)                                                                     \
+  if (dense) return epi ? launch_cfg<__VA_ARGS__, true, true>(plan, dense, feats, W, out, cin, \
+                                                              cout, ep, stream)             \
+                        : launch_cfg<__VA_ARGS__, false, true>(plan, dense, feats, W, out, cin, \
+                                                               cout, ep, stream);           \
+  return epi ? launch_cfg<__VA_ARGS__, true, false>(plan, dense, feats, W, out, cin, cout, ep,    \
+                                                    stream)                                 \
+             : launch_cfg<__VA_ARGS__, false, false>(plan, dense, feats, W, out, cin, cout, ep,   \
+                                                     stream)
+  // tap pairs (K = 3 only): no K = 1 instantiation
+#define SMC_CFG_SPARSE(...)                                                              \
+  if (dense) return SMC_ERR_INVALID;                                                     \
+  return epi ? launch_cfg<__VA_ARGS__, true, false>(plan, dense, feats, W, out, cin, cout, ep,    \
+                                                    stream)                                 \
+             : launch_cfg<__VA_ARGS__, false, false>(plan, dense, feats, W, out, cin, cout, ep,   \
+                                                     stream)
   switch (cfg) {  //            BN  NA NW G WPS NQ        NBUF KS PAIR
     case kCfg256G2: SMC_CFG(256, 9, 2, 2, 4, 3, BF16, 1, 1, false);
     case kCfg256G1: SMC_CFG(256, 9, 2, 1, 4, 3, BF16, 2, 1, false);
     case kCfg256G1K2: SMC_CFG(256, 2, 2, 1, 4, 2, BF16, 2, 2, false);
     case kCfg128G2K2: SMC_CFG(128, 4, 2, 2, 4, 2, BF16, 2, 2, false);
     case kCfg128G1K2: SMC_CFG(128, 4, 2, 1, 4, 2, BF16, 2, 2, false);
-    case kCfg128G1Pair: SMC_CFG(128, 4, 2, 1, 4, 2, BF16, 2, 2, true);
+    case kCfg128G1Pair: SMC_CFG_SPARSE(128, 4, 2, 1, 4, 2, BF16, 2, 2, true);
     case kCfg128G2: SMC_CFG(128, 10, 3, 2, 2, 5, BF16, 2, 1, false);
     case kCfg128G1: SMC_CFG(128, 10, 3, 1, 2, 5, BF16, 2, 1, false);
-    case kCfg64G1Pair: SMC_CFG(64, 5, 2, 1, 2, 5, BF16, 2, 2, true);
+    case kCfg64G1Pair: SMC_CFG_SPARSE(64, 5, 2, 1, 2, 5, BF16, 2, 2, true);
     case kCfg64G2: SMC_CFG(64, 12, 2, 2, 2, 6, BF16, 2, 1, false);
     case kCfg64G1: SMC_CFG(64, 12, 2, 1, 2, 6, BF16, 2, 1, false);
     default: return SMC_ERR_INVALID;
   }
 #undef SMC_CFG
+#undef SMC_CFG_SPARSE
 }
 
 }  // namespace
