@@ -320,6 +320,8 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
   // can be two phases behind, and the abort path can tell which of its loads
   // may still be in flight.
   static_assert(NA % NQ == 0, "every A slot is owned by one gather group");
+  // a stage has at most G units, so each gather group has at most one of them
+  static_assert(NQ >= G, "one unit per gather group and stage");
   // The two MMA warps take the even and odd tiles of an item and meet only at
   // the W ring, so one can run up to NW stages (NW * G units) ahead of the
   // other.  Its wait on an A slot must never be two phases ahead of the
@@ -620,12 +622,23 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
       while (rem && ok) {
         const StageTaps st = next_stage_taps<PAIR>(rem, it.rot);
         for (int kb = 0; kb < kb_per_tap && ok; ++kb) {
+          // the group's unit of this stage, if any (at most one: NQ >= G);
+          // one copy of the code below serves every tile of the group
+          int k = -1;
+          uint32_t my = 0, sl = 0;
 #pragma unroll
-          for (int k = 0; k < G; ++k) {
-            const uint32_t sl = sub_live<G, KS, PAIR>(it, k, st);
-            if (sl == 0u) continue;
-            const uint32_t my = u++;
-            if (int(my % NQ) != grp) continue;
+          for (int t = 0; t < G; ++t) {
+            const uint32_t l = sub_live<G, KS, PAIR>(it, t, st);
+            if (l == 0u) continue;
+            const uint32_t un = u++;
+            if (int(un % NQ) == grp) {
+              k = t;
+              my = un;
+              sl = l;
+            }
+          }
+          if (k < 0) continue;
+          {
             const uint32_t slot = my % NA, ph = (my / NA) & 1;
             const uint32_t dst = a_base + slot * kAUnitBytes;
             if constexpr (DENSE) {
@@ -760,12 +773,22 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
             break;
           }
           const uint64_t bd = bdesc0 + uint64_t(ws) * (kWStage >> 4);
+          // this warp's unit of the stage (its tile, if the tile has the tap);
+          // one copy of the code below serves both tiles
+          int k = -1;
+          uint32_t my = 0, sl = 0;
 #pragma unroll
-          for (int k = 0; k < G; ++k) {
-            const uint32_t sl = sub_live<G, KS, PAIR>(it, k, st);
-            if (sl == 0u) continue;
-            const uint32_t my = u++;
-            if ((uint32_t(k) & 1u) != mine) continue;
+          for (int t = 0; t < G; ++t) {
+            const uint32_t l = sub_live<G, KS, PAIR>(it, t, st);
+            if (l == 0u) continue;
+            const uint32_t un = u++;
+            if ((uint32_t(t) & 1u) == mine) {
+              k = t;
+              my = un;
+              sl = l;
+            }
+          }
+          if (k >= 0) {
             const uint32_t slot = my % NA;
             const bool landed = wt.wait(afull0 + 8 * slot, (my / NA) & 1);
             if (!__all_sync(0xffffffffu, landed)) {
