@@ -47,11 +47,11 @@ DTYPE_NAME = {"f16": "f16", "bf16": "bf16", "f32": "f32"}
 # launch (bytes; profiles/k_conv_tc_*.md).  Cases not captured with the current
 # kernel report null.
 NCU_TRAFFIC: dict = {
-    ("uniform128", 0, "greedy"): 65832192 + 18987520,
-    ("resblock64", 0, "greedy"): 106256896 + 35257856,
-    ("resblock64", 1, "greedy"): 57583104 + 60143360,
-    ("uniform64", 0, "greedy"): 4825856 + 0,
-    ("shells512", 0, "greedy"): 6136039424 + 601306368,
+    ("uniform128", 0, "greedy"): 65752832 + 18645504,
+    ("resblock64", 0, "greedy"): 106253312 + 35474432,
+    ("resblock64", 1, "greedy"): 57569280 + 60423936,
+    ("uniform64", 0, "greedy"): 4822272 + 0,
+    ("shells512", 0, "greedy"): 6124230144 + 601768192,
     ("tiny16", 0, "greedy"): 116480 + 0,
 }
 # fp32 features run on the CUDA cores with fp64 accumulation: the ALU bound is
