@@ -322,6 +322,9 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
   static_assert(NA % NQ == 0, "every A slot is owned by one gather group");
   // a stage has at most G units, so each gather group has at most one of them
   static_assert(NQ >= G, "one unit per gather group and stage");
+  // the first four gather warps (consecutive warps: one per tensor-memory lane
+  // quarter) store half of the CTA's last item
+  static_assert(NQ * WPS >= 4, "four gather warps help store the last item");
   // The two MMA warps take the even and odd tiles of an item and meet only at
   // the W ring, so one can run up to NW stages (NW * G units) ahead of the
   // other.  Its wait on an A slot must never be two phases ahead of the
