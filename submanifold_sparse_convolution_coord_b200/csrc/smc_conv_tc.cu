@@ -116,57 +116,72 @@ __device__ __forceinline__ float half_to_float(uint16_t h) {
     return __half2float(__ushort_as_half(h));
 }
 
-__device__ __forceinline__ float act_apply(float v, int act) {
-  switch (act) {
-    case SMC_ACT_RELU:
-      return fmaxf(v, 0.f);
-    case SMC_ACT_SILU:
-      return v / (1.f + expf(-v));
-    case SMC_ACT_GELU:
-      return 0.5f * v * (1.f + erff(v * 0.7071067811865476f));
-    default:
-      return v;
+// Adds 32 fp16/bf16 values (four 16-byte words, element order) to v.
+template <bool BF16>
+__device__ __forceinline__ void add_halves(uint32_t (&v)[32], const uint4 (&h)[4]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t w[4] = {h[q].x, h[q].y, h[q].z, h[q].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      v[8 * q + 2 * e] = __float_as_uint(__uint_as_float(v[8 * q + 2 * e]) +
+                                         half_to_float<BF16>(uint16_t(w[e] & 0xFFFFu)));
+      v[8 * q + 2 * e + 1] = __float_as_uint(__uint_as_float(v[8 * q + 2 * e + 1]) +
+                                             half_to_float<BF16>(uint16_t(w[e] >> 16)));
+    }
   }
 }
 
-// act(acc + bias) + residual on 32 consecutive columns of one output row (in
-// place, fp32), before the one rounding to the output dtype.
+// act(acc + bias) on 32 consecutive columns of one output row, in fp32.  The
+// activation is chosen once per call, and SiLU uses the fast exponential and
+// division (their error, a few fp32 ulps, is far below the output's one
+// rounding; for very negative x the divisor is infinite and the result the
+// limit 0).
 template <bool BF16>
-__device__ __forceinline__ void apply_epilogue(uint32_t (&v)[32], const ConvArgs& a, int64_t row,
-                                               int col) {
+__device__ __forceinline__ void bias_activation(uint32_t (&v)[32], const ConvArgs& a, int col) {
   if (a.bias) {
     const uint4* b4 = reinterpret_cast<const uint4*>(a.bias + col);
+    uint4 b[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const uint4 u = __ldg(b4 + q);
-      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        v[8 * q + 2 * e] = __float_as_uint(__uint_as_float(v[8 * q + 2 * e]) +
-                                           half_to_float<BF16>(uint16_t(w[e] & 0xFFFFu)));
-        v[8 * q + 2 * e + 1] = __float_as_uint(__uint_as_float(v[8 * q + 2 * e + 1]) +
-                                               half_to_float<BF16>(uint16_t(w[e] >> 16)));
-      }
-    }
+    for (int q = 0; q < 4; ++q) b[q] = __ldg(b4 + q);
+    add_halves<BF16>(v, b);
   }
-  if (a.act != SMC_ACT_NONE) {
+  switch (a.act) {
+    case SMC_ACT_RELU:
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(act_apply(__uint_as_float(v[i]), a.act));
-  }
-  if (a.residual) {
-    const uint4* r4 = reinterpret_cast<const uint4*>(a.residual + row * a.cout + col);
+      for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(fmaxf(__uint_as_float(v[i]), 0.f));
+      break;
+    case SMC_ACT_SILU:
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const uint4 u = r4[q];
-      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        v[8 * q + 2 * e] = __float_as_uint(__uint_as_float(v[8 * q + 2 * e]) +
-                                           half_to_float<BF16>(uint16_t(w[e] & 0xFFFFu)));
-        v[8 * q + 2 * e + 1] = __float_as_uint(__uint_as_float(v[8 * q + 2 * e + 1]) +
-                                               half_to_float<BF16>(uint16_t(w[e] >> 16)));
+      for (int i = 0; i < 32; ++i) {
+        const float x = __uint_as_float(v[i]);
+        v[i] = __float_as_uint(__fdividef(x, 1.f + __expf(-x)));
       }
-    }
+      break;
+    case SMC_ACT_GELU:
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float x = __uint_as_float(v[i]);
+        v[i] = __float_as_uint(0.5f * x * (1.f + erff(x * 0.7071067811865476f)));
+      }
+      break;
+    default:
+      break;
+  }
+}
+
+// The residual's 32 columns of one output row (zeros when there is none or
+// the row is padding), loaded one chunk ahead of their use.
+template <bool BF16>
+__device__ __forceinline__ void load_residual(uint4 (&r)[4], const ConvArgs& a, int32_t row,
+                                              int col) {
+  if (a.residual && row >= 0) {
+    const uint4* r4 = reinterpret_cast<const uint4*>(a.residual + int64_t(row) * a.cout + col);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) r[q] = __ldg(r4 + q);
+  } else {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) r[q] = make_uint4(0u, 0u, 0u, 0u);
   }
 }
 
@@ -458,15 +473,27 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
     for (int k = 0; k < G; ++k) {
       if (it.mask[k] == 0) continue;  // past the last tile
       uint16_t* dst = args.out + int64_t(orow[k] < 0 ? 0 : orow[k]) * args.cout + it.n0;
+      uint4 res[4];  // the fused epilogue's residual, one chunk ahead
+      if constexpr (EPI) load_residual<BF16>(res, args, orow[k], it.n0 + cc0 * 32);
 #pragma unroll 1
       for (int cc = cc0; cc < cc1; ++cc) {
         uint32_t v[32];
         tmem_ld_x32(tmem + (uint32_t(quarter * 32) << 16) + (a * G + k) * BN + uint32_t(cc * 32),
                     v);
+        if constexpr (EPI) {
+          // act(acc + bias) + residual, before the one rounding
+          uint4 cur[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) cur[q] = res[q];
+          if (cc + 1 < cc1) load_residual<BF16>(res, args, orow[k], it.n0 + (cc + 1) * 32);
+          if (orow[k] >= 0) {
+            bias_activation<BF16>(v, args, it.n0 + cc * 32);
+            add_halves<BF16>(v, cur);
+          }
+        }
         if constexpr (kStaged) {
           // this lane's row piece into the warp's staging rows, then each
           // store writes 64-byte pieces of 8 rows (4 lanes per row)
-          if (EPI && orow[k] >= 0) apply_epilogue<BF16>(v, args, orow[k], it.n0 + cc * 32);
           uint4* mine_row = reinterpret_cast<uint4*>(st_rows + lane * kStageRowBytes);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -491,7 +518,6 @@ k_conv_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUte
           continue;
         }
         if (orow[k] >= 0) {
-          if (EPI) apply_epilogue<BF16>(v, args, orow[k], it.n0 + cc * 32);
           uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
